@@ -1,0 +1,163 @@
+"""Seeded synthetic inputs for the MoE layer forward.
+
+Shared by the tests, ``bench.py``, ``__graft_entry__.smoke()`` and the CPU
+oracle.  This module draws random numbers and lays them out; it contains
+none of the layer's arithmetic (no gating, sorting, FFN or combine).
+
+Recipes (workload shapes from the MoE Align & Sort article's DeepSeek-V3
+workloads -- E=256, top-8 -- and the aiter a8w8 issue's hidden 7168 /
+inter 2048 shape):
+
+* activations ``x`` ~ N(0, 1), rounded to bf16 by torch's cast;
+* expert weights ~ N(0, 0.02), generated directly in the library's
+  K-contiguous layout ``w13 [E, 2I, H]`` (rows 0..I-1 gate, I..2I-1 up) and
+  ``w2 [E, H, I]``; the entries are i.i.d., so the layout is only a choice
+  of which random number lands where;
+* FP8 weights: model preparation, not part of the forward pass.  Per output
+  channel the fp32 draw is divided by ``amax / 448`` and cast to E4M3FN by
+  torch (after clamping to +-448); the codes and the fp32 scales are the
+  layer's parameters and both sides read the same bytes;
+* router logits: ``x @ Wr`` with Wr ~ N(0, 0.02) in fp32 for the tiny
+  layer, i.i.d. N(0, 1) otherwise (so the top-k set is a uniformly random
+  k-subset); the skewed variant adds a per-expert N(0, 1) bias;
+* align-only ids: k distinct experts per token drawn one after another
+  without replacement from Zipf(s) popularity over a seeded permutation of
+  the experts (Gumbel-top-k, which has exactly that law), or uniformly.
+
+Large weights are drawn on the target device with a seeded
+``torch.Generator`` on that device.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import numpy as np
+import torch
+
+SEED_BASE = 0x5EED0000
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    bm: int
+    a8w8: bool = False
+    bias: bool = False
+    router: str = "normal"      # "normal": logits ~ N(0,1); "linear": x @ Wr
+    seed: int = SEED_BASE
+
+    def with_(self, **kw) -> "MoEConfig":
+        return replace(self, **kw)
+
+
+CONFIGS = {
+    # tiny layer used for full parity
+    "tiny": MoEConfig("tiny", T=64, H=256, I=128, E=8, k=2, bm=16,
+                      router="linear", seed=SEED_BASE + 0),
+    # Mixtral-shaped prefill, bf16
+    "mixtral": MoEConfig("mixtral", T=4096, H=4096, I=14336, E=8, k=2, bm=128,
+                         seed=SEED_BASE + 2),
+    # DeepSeek-V3-shaped prefill (uniform routing); a8w8 / bias / bm variants
+    "deepseek": MoEConfig("deepseek", T=2048, H=7168, I=2048, E=256, k=8, bm=64,
+                          seed=SEED_BASE + 3),
+    # decode sweep, FP8 a8w8 (T in 1, 16, 64, 256)
+    "decode": MoEConfig("decode", T=64, H=7168, I=2048, E=256, k=8, bm=16,
+                        a8w8=True, seed=SEED_BASE + 4),
+}
+
+ALIGN_CONFIG = dict(T=16384, E=256, k=8, bm=64, zipf_s=1.0, seed=SEED_BASE + 1)
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def normal(shape, std, seed, device="cpu", dtype=torch.float32):
+    g = _gen(device, seed)
+    t = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    return (t * std).to(dtype)
+
+
+def fp8_weights(E, rows, cols, std, seed, device="cpu"):
+    """E4M3FN codes [E, rows, cols] and fp32 per-row scales [E, rows]."""
+    codes = torch.empty(E, rows, cols, dtype=torch.float8_e4m3fn, device=device)
+    scales = torch.empty(E, rows, dtype=torch.float32, device=device)
+    g = _gen(device, seed)
+    for e in range(E):
+        w = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32) * std
+        amax = w.abs().amax(dim=1)
+        s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        codes[e] = (w / s[:, None]).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn)
+        scales[e] = s
+    return codes, scales
+
+
+def make_layer(cfg: MoEConfig, device="cpu", weights=True):
+    """All inputs of one MoE layer forward for ``cfg``.
+
+    Returns a dict with x (bf16 [T,H]), logits (f32 [T,E]), bias (f32 [E] or
+    None) and, when ``weights``: w13/w2 (bf16) or w13_q/w13_s/w2_q/w2_s
+    (float8_e4m3fn codes + f32 scales).
+    """
+    T, H, I, E = cfg.T, cfg.H, cfg.I, cfg.E
+    s = cfg.seed
+    d = {}
+    d["x"] = normal((T, H), 1.0, s * 16 + 1, device, torch.bfloat16)
+    if cfg.router == "linear":
+        wr = normal((H, E), 0.02, s * 16 + 2, device)
+        d["logits"] = (d["x"].float() @ wr).contiguous()
+    else:
+        d["logits"] = normal((T, E), 1.0, s * 16 + 3, device)
+    d["bias"] = normal((E,), 1.0, s * 16 + 4, device) if cfg.bias else None
+    if weights:
+        if cfg.a8w8:
+            d["w13_q"], d["w13_s"] = fp8_weights(E, 2 * I, H, 0.02, s * 16 + 5, device)
+            d["w2_q"], d["w2_s"] = fp8_weights(E, H, I, 0.02, s * 16 + 6, device)
+        else:
+            d["w13"] = normal((E, 2 * I, H), 0.02, s * 16 + 5, device, torch.bfloat16)
+            d["w2"] = normal((E, H, I), 0.02, s * 16 + 6, device, torch.bfloat16)
+    return d
+
+
+def align_ids(T, E, k, seed, dist="zipf", zipf_s=1.0):
+    """int32 [T, k]: k distinct experts per token.
+
+    ``zipf``: popularity of the expert at rank r (r = 1..E, ranks assigned by
+    a seeded permutation) is proportional to r**-s; the k experts are drawn
+    one after another without replacement, renormalising each time.  The
+    Gumbel-top-k construction (keys log p + Gumbel noise, take the k largest
+    in descending order) has exactly that distribution.  ``uniform``: every
+    expert equally likely.
+    """
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(E)
+    if dist == "zipf":
+        p_rank = np.arange(1, E + 1, dtype=np.float64) ** (-zipf_s)
+        logp = np.empty(E)
+        logp[perm] = np.log(p_rank)            # expert perm[r] has rank r+1
+    elif dist == "uniform":
+        logp = np.zeros(E)
+    else:
+        raise ValueError(dist)
+    keys = logp[None, :] + rng.gumbel(size=(T, E))
+    top = np.argsort(-keys, axis=1, kind="stable")[:, :k]
+    return top.astype(np.int32)
+
+
+def to_numpy(t):
+    """float64 / int numpy view of a (possibly device, bf16 or fp8) tensor."""
+    if t is None:
+        return None
+    t = t.detach().cpu()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.float().numpy().astype(np.float64)
+    return t.numpy()
