@@ -1,0 +1,221 @@
+/*
+ * moe_b200.h -- C ABI of the single-GPU MoE layer forward for NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer, as the pages define it (MoE Align & Sort article on
+ * dignews.cc, opening definition of the MoE layer and its "FasterTransformer",
+ * "Megatron", "CK" and D-C-P sections; aiter issue 1248 "[Feature]: Add more
+ * configuration options for MoE assembly kernels", "Suggestion Description"):
+ *
+ *   gate     : softmax top-k over E expert logits per token, weights
+ *              renormalised over the k chosen experts          (moe_topk_gate)
+ *   align    : counting sort of the T*k (token, choice) slots by expert,
+ *              each expert's segment padded to a multiple of block_size
+ *                                                             (moe_align_sort)
+ *   FFN      : per block of sorted slots, the owning expert's gated FFN
+ *              h = silu(x Wg^T) * (x Wu^T), y = h Wd^T, in bf16 or with
+ *              per-token FP8 E4M3 activations and per-channel FP8 weights
+ *                                                            (moe_grouped_ffn)
+ *   combine  : out[t] = sum_j w[t,j] * y[t*k+j]                  (moe_combine)
+ *   all four : moe_forward
+ *
+ * Conventions (every entry point):
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise.  The
+ *     caller owns every buffer and the stream; the library allocates no
+ *     device memory and keeps no per-call state between calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and stream-ordered; none synchronises
+ *     the host.
+ *   - Arguments are validated synchronously; a bad argument returns an error
+ *     and launches nothing.  Errors found on the device (an expert id out of
+ *     range, a bounded wait that ran out) are OR-ed into *dev_status (bit
+ *     flags MOE_DEV_*) when dev_status is non-NULL; the caller reads it after
+ *     synchronising.  With dev_status NULL they are dropped and the outputs
+ *     are unspecified.
+ *   - Layouts are row-major and contiguous.  Flat slot i = t*k + j names
+ *     token t's j-th choice.
+ *   - Requires an sm_100a device.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, k > E, ...     */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but not handled (e.g. H % 128 != 0)   */
+  MOE_ERR_WORKSPACE = 3,     /* workspace smaller than the size query says  */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (see moe_last_cuda_error) */
+  MOE_ERR_DEVICE = 5         /* no sm_100 device current                    */
+} moe_status_t;
+
+typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2 } moe_dtype_t;
+
+/* Device-side status bits (OR-ed into *dev_status). */
+#define MOE_DEV_BAD_EXPERT_ID 0x1  /* an expert id outside [0, E): slot skipped */
+#define MOE_DEV_TIMEOUT       0x2  /* a bounded wait ran out; outputs unspecified */
+#define MOE_DEV_BAD_PLAN      0x4  /* routing metadata inconsistent with sizes  */
+
+/* Human-readable name of a status code.  Host only; never fails. */
+MOE_API const char* moe_status_string(int status);
+/* Text of the last CUDA error seen by this thread inside the library. */
+MOE_API const char* moe_last_cuda_error(void);
+/* ABI version (major*100 + minor). */
+MOE_API int moe_version(void);
+
+/* ---------------------------------------------------------------------------
+ * moe_topk_gate -- softmax top-k gating.
+ * Passage: MoE Align & Sort article, "FasterTransformer" (moe_softmax +
+ * moe_top_k fused as topk_gating_softmax; "biased" variant) and the opening
+ * definition (Top-K gating scores, a gating bias in DeepSeek V3).
+ *
+ *   logits   f32 [T, E]   router logits (the router GEMM is the caller's)
+ *   bias     f32 [E]      nullable; added to the logits in fp32 before both
+ *                         the selection and the softmax
+ *   topk_ids i32 [T, k]   out: chosen experts, by descending (biased) logit;
+ *                         equal logits go to the lower expert index
+ *   topk_w   f32 [T, k]   out: softmax(l)[chosen] / sum(softmax(l)[chosen])
+ * Limits: 0 <= T, 1 <= E <= 1024, 1 <= k <= min(E, 32).  Logits must be
+ * finite.  Errors: MOE_ERR_INVALID_ARG on a bad size or NULL output.
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_topk_gate(const float* logits, const float* bias, int T, int E, int k,
+                           int32_t* topk_ids, float* topk_w, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_align_sort -- block-aligned MoE Align & Sort.
+ * Passage: MoE Align & Sort article, the D-C-P section (distributed
+ * concurrent counting; unaligned local cumsum, merge, aligned global cumsum;
+ * parallel placement) and the paragraph on aligned sorting for Group GEMM.
+ *
+ *   topk_ids   i32 [T*k]  expert of every flat slot
+ *   sorted_ids i32 [P]    out: slots grouped by expert (ascending expert,
+ *                         ascending slot inside an expert), every expert's
+ *                         segment padded with the sentinel T*k to a multiple
+ *                         of block_size; experts with no slot get no block.
+ *                         Entries [num_post, P) are not written.
+ *   expert_ids i32 [NB]   out: expert owning each block of block_size
+ *                         entries; entries [num_post/block_size, NB) are not
+ *                         written.
+ *   num_post   i32 [1]    out: padded length = sum_e ceil(c_e/bs)*bs
+ *   ws, ws_bytes          device workspace of at least the size
+ *                         moe_align_sort_sizes returns; contents on entry are
+ *                         irrelevant.
+ * P = T*k + E*(block_size-1), NB = ceil(P / block_size) (host values from
+ * moe_align_sort_sizes).  Limits: 1 <= E <= 1024, 1 <= block_size <= 1024,
+ * T*k < 2^31 - 1.  Out-of-range ids are skipped and flagged with
+ * MOE_DEV_BAD_EXPERT_ID.  The kernel runs as one cooperative grid with a
+ * bounded grid-wide wait (MOE_DEV_TIMEOUT if it runs out).
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_align_sort_sizes(int T, int k, int E, int block_size,
+                                  size_t* P, size_t* NB, size_t* ws_bytes);
+MOE_API moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int k, int E, int block_size,
+                            int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_post,
+                            void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_ffn -- gated grouped expert FFN over the sorted slots.
+ * Passage: MoE Align & Sort article, opening definition (expert FFNs on the
+ * chosen tokens computed by a Group GEMM) and "AITER" (the grouped GEMM
+ * multiplies each expert's FFN weights with a block of token hidden states);
+ * aiter issue 1248, "Suggestion Description" (g1u1 SiLU, per-token FP8
+ * activations with bf16 in/out); GC-MoE abstract (fused SwiGLU and
+ * requantisation between the two GEMMs).
+ *
+ * For every sorted row r < num_post with slot s = sorted_ids[r] != T*k and
+ * expert e = expert_ids[r / block_size], token t = s / k:
+ *   BF16:  g = Wg[e] x_t, u = Wu[e] x_t (fp32 accumulation),
+ *          h = bf16(silu(g) * u), y_s = Wd[e] h
+ *   FP8:   (q_x, s_x) = e4m3 per-token quantisation of x_t (s = amax/448),
+ *          g = (Wg_q[e] q_x) * s_x * w13_scale[e], u likewise,
+ *          h = bf16(silu(g) * u), (q_h, s_h) = per-row requantisation,
+ *          y_s = (Wd_q[e] q_h) * s_h * w2_scale[e]
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int T, H, I, E, k, block_size;
+  int wdtype;                 /* MOE_BF16 or MOE_FP8_E4M3                       */
+  const void* x;              /* bf16 [T, H]                                     */
+  const void* w13;            /* [E, 2I, H]: rows 0..I-1 gate, I..2I-1 up;
+                                 bf16, or E4M3 codes when wdtype is FP8          */
+  const float* w13_scale;     /* f32 [E, 2I] per output channel (FP8 only)       */
+  const void* w2;             /* [E, H, I] bf16 or E4M3 codes                    */
+  const float* w2_scale;      /* f32 [E, H] (FP8 only)                           */
+  const int32_t* sorted_ids;  /* [P]  from moe_align_sort                        */
+  const int32_t* expert_ids;  /* [NB] from moe_align_sort                        */
+  const int32_t* num_post;    /* [1]  from moe_align_sort                        */
+  int tile_tokens;            /* tokens per GEMM tile: 0 = automatic, else one
+                                 of 16, 32, 64, 128, 256                          */
+} moe_ffn_args;
+
+/* Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32,
+ * 1 <= block_size <= 1024; device pointers 16-byte aligned. */
+MOE_API moe_status_t moe_ffn_workspace(const moe_ffn_args* args, size_t* ws_bytes);
+/*   y  f32 [T*k, H]  out: per-slot expert output y_s (rows of slots that were
+ *                    skipped are not written) */
+MOE_API moe_status_t moe_grouped_ffn(const moe_ffn_args* args, float* y, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- top-k weighted combine (unpermute).
+ * Passage: MoE Align & Sort article, "Megatron" (unpermute) and
+ * "FasterTransformer" (permute before the group GEMM).
+ *   y       f32 [T*k, H];  topk_w f32 [T, k]
+ *   out     [T, H] in out_dtype (MOE_BF16 or MOE_F32):
+ *           out[t] = sum_j topk_w[t,j] * y[t*k+j], summed in fp32 in
+ *           ascending j, rounded once.
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int H,
+                         void* out, int out_dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_forward -- gate, align & sort, grouped FFN and combine in one call.
+ * The combine is fused into the down projection (fp32 atomic accumulation,
+ * so the summation order over the k choices is not fixed).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int T, H, I, E, k, block_size;
+  int wdtype;                 /* MOE_BF16 or MOE_FP8_E4M3                 */
+  int out_dtype;              /* MOE_BF16 or MOE_F32                      */
+  const void* x;              /* bf16 [T, H]                              */
+  const float* logits;        /* f32 [T, E]                               */
+  const float* bias;          /* f32 [E], nullable                        */
+  const void* w13;            /* as in moe_ffn_args                       */
+  const float* w13_scale;
+  const void* w2;
+  const float* w2_scale;
+  void* out;                  /* [T, H] out_dtype                         */
+  int32_t* topk_ids;          /* nullable: routing also written here [T,k] */
+  float* topk_w;              /* nullable [T,k]                           */
+  int tile_tokens;            /* as in moe_ffn_args                       */
+} moe_forward_args;
+
+MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);
+MOE_API moe_status_t moe_forward(const moe_forward_args* args, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics.
+ * moe_test_wait_timeout runs the grid-wide wait of moe_align_sort on a
+ * barrier that can never fill (it expects one more arrival than the grid
+ * has) with the given limit in nanoseconds, so that the timeout path can be
+ * exercised without a fault: it must OR MOE_DEV_TIMEOUT into *dev_status and
+ * return.  ws: at least 256 bytes of device memory.
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_test_wait_timeout(void* ws, int32_t* dev_status, long long timeout_ns,
+                                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

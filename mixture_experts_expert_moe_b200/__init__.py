@@ -1,0 +1,264 @@
+"""Python binding of the B200 MoE layer-forward library (libmoe_b200.so).
+
+Argument marshalling only: every step of the forward runs in the CUDA
+kernels behind the C ABI declared in ``include/moe_b200.h``.  PyTorch is used
+for device memory (workspaces and outputs are torch tensors) and for the
+current CUDA stream.  There is no CPU fallback: if the shared library is not
+built, importing the ops raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_BF16, MOE_FP8_E4M3, MOE_F32 = 0, 1, 2
+MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN = 0x1, 0x2, 0x4
+
+EXPORTED = [
+    "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
+    "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
+    "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
+]
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+class FfnArgs(ctypes.Structure):
+    _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i),
+                ("wdtype", _i), ("x", _vp), ("w13", _vp), ("w13_scale", _vp), ("w2", _vp),
+                ("w2_scale", _vp), ("sorted_ids", _vp), ("expert_ids", _vp), ("num_post", _vp),
+                ("tile_tokens", _i)]
+
+
+class ForwardArgs(ctypes.Structure):
+    _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i),
+                ("wdtype", _i), ("out_dtype", _i), ("x", _vp), ("logits", _vp), ("bias", _vp),
+                ("w13", _vp), ("w13_scale", _vp), ("w2", _vp), ("w2_scale", _vp), ("out", _vp),
+                ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i)]
+
+
+_LIB = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe_b200.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build it with `python -m mixture_experts_expert_moe_b200.build_lib`")
+        lib = ctypes.CDLL(path)
+        sz = ctypes.POINTER(ctypes.c_size_t)
+        sigs = {
+            "moe_status_string": (ctypes.c_char_p, [_i]),
+            "moe_last_cuda_error": (ctypes.c_char_p, []),
+            "moe_version": (_i, []),
+            "moe_topk_gate": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+            "moe_align_sort_sizes": (_i, [_i, _i, _i, _i, sz, sz, sz]),
+            "moe_align_sort": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]),
+            "moe_ffn_workspace": (_i, [ctypes.POINTER(FfnArgs), sz]),
+            "moe_grouped_ffn": (_i, [ctypes.POINTER(FfnArgs), _vp, _vp, ctypes.c_size_t, _vp, _vp]),
+            "moe_combine": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp]),
+            "moe_forward_workspace": (_i, [ctypes.POINTER(ForwardArgs), sz]),
+            "moe_forward": (_i, [ctypes.POINTER(ForwardArgs), _vp, ctypes.c_size_t, _vp, _vp]),
+            "moe_test_wait_timeout": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        lib = load_library()
+        msg = lib.moe_status_string(status).decode()
+        cuda = lib.moe_last_cuda_error().decode()
+        raise MoEError(f"{what}: {msg}" + (f" ({cuda})" if cuda and status == 4 else ""))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dev_status(dev_status, device):
+    if dev_status is None:
+        return None
+    assert dev_status.dtype == torch.int32 and dev_status.device == device
+    return _ptr(dev_status)
+
+
+def _wdtype(w):
+    if w.dtype == torch.bfloat16:
+        return MOE_BF16
+    if w.dtype in (torch.float8_e4m3fn, torch.uint8):
+        return MOE_FP8_E4M3
+    raise TypeError(f"unsupported weight dtype {w.dtype}")
+
+
+# ---------------------------------------------------------------------------
+# ops
+# ---------------------------------------------------------------------------
+
+def topk_gate(logits: torch.Tensor, k: int, bias: torch.Tensor | None = None):
+    """Softmax top-k gating: returns (ids int32 [T,k], weights f32 [T,k])."""
+    lib = load_library()
+    assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous()
+    T, E = logits.shape
+    ids = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    _check(lib.moe_topk_gate(_ptr(logits), _ptr(bias), T, E, k, _ptr(ids), _ptr(w),
+                             _stream(logits.device)), "moe_topk_gate")
+    return ids, w
+
+
+def align_sort_sizes(T: int, k: int, E: int, block_size: int):
+    lib = load_library()
+    P, NB, ws = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.moe_align_sort_sizes(T, k, E, block_size, ctypes.byref(P), ctypes.byref(NB),
+                                    ctypes.byref(ws)), "moe_align_sort_sizes")
+    return P.value, NB.value, ws.value
+
+
+def align_sort(topk_ids: torch.Tensor, E: int, block_size: int, dev_status=None, ws=None, out=None):
+    """Block-aligned align&sort.  Returns (sorted_ids [P], expert_ids [NB],
+    num_post [1]); only the first num_post / num_post//block_size entries are
+    defined."""
+    lib = load_library()
+    assert topk_ids.is_cuda and topk_ids.dtype == torch.int32 and topk_ids.is_contiguous()
+    T, k = topk_ids.shape
+    P, NB, wsb = align_sort_sizes(T, k, E, block_size)
+    dev = topk_ids.device
+    if out is None:
+        out = (torch.empty(P, dtype=torch.int32, device=dev), torch.empty(NB, dtype=torch.int32, device=dev),
+               torch.empty(1, dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    s, b, n = out
+    _check(lib.moe_align_sort(_ptr(topk_ids), T, k, E, block_size, _ptr(s), _ptr(b), _ptr(n), _ptr(ws),
+                              ws.numel(), _dev_status(dev_status, dev), _stream(dev)), "moe_align_sort")
+    return s, b, n
+
+
+def _ffn_args(x, w13, w2, sorted_ids, expert_ids, num_post, T, k, E, block_size, w13_scale, w2_scale,
+              tile_tokens):
+    H = x.shape[1]
+    I = w13.shape[1] // 2
+    a = FfnArgs(T=T, H=H, I=I, E=E, k=k, block_size=block_size, wdtype=_wdtype(w13),
+                x=x.data_ptr(), w13=w13.data_ptr(), w2=w2.data_ptr(),
+                w13_scale=None if w13_scale is None else w13_scale.data_ptr(),
+                w2_scale=None if w2_scale is None else w2_scale.data_ptr(),
+                sorted_ids=sorted_ids.data_ptr(), expert_ids=expert_ids.data_ptr(),
+                num_post=num_post.data_ptr(), tile_tokens=tile_tokens)
+    return a
+
+
+def grouped_ffn(x, w13, w2, sorted_ids, expert_ids, num_post, k, block_size, w13_scale=None, w2_scale=None,
+                tile_tokens=0, dev_status=None, y=None, ws=None):
+    """Per-slot expert FFN output y f32 [T*k, H] over align&sort's outputs."""
+    lib = load_library()
+    T, H = x.shape
+    E = w13.shape[0]
+    a = _ffn_args(x, w13, w2, sorted_ids, expert_ids, num_post, T, k, E, block_size, w13_scale, w2_scale,
+                  tile_tokens)
+    nbytes = ctypes.c_size_t()
+    _check(lib.moe_ffn_workspace(ctypes.byref(a), ctypes.byref(nbytes)), "moe_ffn_workspace")
+    if ws is None:
+        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty(T * k, H, dtype=torch.float32, device=x.device)
+    _check(lib.moe_grouped_ffn(ctypes.byref(a), _ptr(y), _ptr(ws), ws.numel(),
+                               _dev_status(dev_status, x.device), _stream(x.device)), "moe_grouped_ffn")
+    return y
+
+
+def combine(y: torch.Tensor, topk_w: torch.Tensor, out_dtype=torch.bfloat16, out=None):
+    """out[t] = sum_j w[t,j] * y[t*k+j]."""
+    lib = load_library()
+    T, k = topk_w.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=out_dtype, device=y.device)
+    od = MOE_BF16 if out.dtype == torch.bfloat16 else MOE_F32
+    _check(lib.moe_combine(_ptr(y), _ptr(topk_w), T, k, H, _ptr(out), od, _stream(y.device)), "moe_combine")
+    return out
+
+
+class MoELayer:
+    """One MoE layer forward through ``moe_forward`` with a reusable workspace.
+
+    Weights: ``w13 [E, 2I, H]`` (gate rows then up rows) and ``w2 [E, H, I]``,
+    bf16, or float8_e4m3fn codes with f32 per-row scales ``w13_scale [E, 2I]``
+    and ``w2_scale [E, H]``.
+    """
+
+    def __init__(self, w13, w2, k, block_size, w13_scale=None, w2_scale=None, out_dtype=torch.bfloat16,
+                 tile_tokens=0):
+        self.w13, self.w2, self.k, self.block_size = w13, w2, k, block_size
+        self.w13_scale, self.w2_scale = w13_scale, w2_scale
+        self.out_dtype, self.tile_tokens = out_dtype, tile_tokens
+        self.E, twoI, self.H = w13.shape
+        self.I = twoI // 2
+        self._ws = None
+
+    def _args(self, x, logits, bias, out, ids, w):
+        T = x.shape[0]
+        return ForwardArgs(
+            T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
+            wdtype=_wdtype(self.w13), out_dtype=MOE_BF16 if out.dtype == torch.bfloat16 else MOE_F32,
+            x=x.data_ptr(), logits=logits.data_ptr(), bias=None if bias is None else bias.data_ptr(),
+            w13=self.w13.data_ptr(), w13_scale=None if self.w13_scale is None else self.w13_scale.data_ptr(),
+            w2=self.w2.data_ptr(), w2_scale=None if self.w2_scale is None else self.w2_scale.data_ptr(),
+            out=out.data_ptr(), topk_ids=None if ids is None else ids.data_ptr(),
+            topk_w=None if w is None else w.data_ptr(), tile_tokens=self.tile_tokens)
+
+    def workspace_bytes(self, T):
+        lib = load_library()
+        a = ForwardArgs(T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
+                        wdtype=_wdtype(self.w13),
+                        out_dtype=MOE_BF16 if self.out_dtype == torch.bfloat16 else MOE_F32,
+                        tile_tokens=self.tile_tokens)
+        n = ctypes.c_size_t()
+        _check(lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)), "moe_forward_workspace")
+        return n.value
+
+    def __call__(self, x, logits, bias=None, out=None, topk_ids=None, topk_w=None, dev_status=None):
+        lib = load_library()
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, self.H, dtype=self.out_dtype, device=x.device)
+        need = self.workspace_bytes(T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=x.device)
+        a = self._args(x, logits, bias, out, topk_ids, topk_w)
+        _check(lib.moe_forward(ctypes.byref(a), _ptr(self._ws), self._ws.numel(),
+                               _dev_status(dev_status, x.device), _stream(x.device)), "moe_forward")
+        return out
+
+
+def run_wait_timeout_check(timeout_ns: int, device="cuda"):
+    """Run the bounded grid-wide wait on a barrier that never fills; returns
+    the device status word (MOE_DEV_TIMEOUT expected)."""
+    lib = load_library()
+    ws = torch.zeros(64, dtype=torch.int32, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib.moe_test_wait_timeout(_ptr(ws), _ptr(st), int(timeout_ns), _stream(torch.device(device))),
+           "moe_test_wait_timeout")
+    torch.cuda.synchronize()
+    return int(st.item())

@@ -1,0 +1,396 @@
+// Host side of the C ABI declared in include/moe_b200.h: argument checks,
+// workspace carving and kernel launches.  No device memory is allocated and
+// no call synchronises the host.
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+moe_status_t cuda_fail(cudaError_t e, const char* where) {
+  char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+  g_last_cuda_error = buf;
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CU(call)                                          \
+  do {                                                        \
+    cudaError_t _e = (call);                                  \
+    if (_e != cudaSuccess) return cuda_fail(_e, #call);       \
+  } while (0)
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Carver {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  }
+};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+moe_status_t check_device() {
+  int dev = 0, major = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  return major == 10 ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+// ---------------------------------------------------------------------------
+// align & sort
+// ---------------------------------------------------------------------------
+constexpr int kMaxAlignCtas = 1024;
+constexpr int kMinSlotsPerCta = 4096;
+
+bool align_args_ok(int T, int k, int E, int bm) {
+  return T >= 0 && k >= 1 && E >= 1 && E <= 1024 && bm >= 1 && bm <= 1024 &&
+         (long long)T * k + (long long)E * (bm - 1) < 0x7FFFFFFFLL;
+}
+
+size_t align_ws_bytes(int E) { return 256 + (size_t)kMaxAlignCtas * E * sizeof(int32_t); }
+
+moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t* sorted, int32_t* expert_ids,
+                       int32_t* num_post, void* ws, int32_t* status, cudaStream_t stream) {
+  const int N = T * k;
+  int err = 0;
+  const int max_ctas = moe::align_max_ctas(E, &err);
+  if (err) return cuda_fail((cudaError_t)err, "align occupancy");
+  if (max_ctas < 1) return MOE_ERR_UNSUPPORTED;
+  const int per_cta_unit = 32 * 16;  // warps x lanes
+  int grid = (N + kMinSlotsPerCta - 1) / kMinSlotsPerCta;
+  grid = grid < 1 ? 1 : grid;
+  grid = grid > max_ctas ? max_ctas : grid;
+  grid = grid > kMaxAlignCtas ? kMaxAlignCtas : grid;
+  int chunk = (N + grid - 1) / grid;
+  chunk = (chunk + per_cta_unit - 1) / per_cta_unit * per_cta_unit;
+  if (chunk < per_cta_unit) chunk = per_cta_unit;
+  grid = N > 0 ? (N + chunk - 1) / chunk : 1;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  moe::AlignParams p;
+  p.ids = ids;
+  p.N = N;
+  p.E = E;
+  p.bm = bm;
+  p.chunk = chunk;
+  p.sorted = sorted;
+  p.expert_ids = expert_ids;
+  p.num_post = num_post;
+  p.barrier = reinterpret_cast<int*>(w);
+  p.hist = reinterpret_cast<int32_t*>(w + 256);
+  p.status = status;
+  p.timeout_ns = moe::kDefaultTimeoutNs;
+  p.expected = grid;
+  MOE_CU(cudaMemsetAsync(p.barrier, 0, sizeof(int), stream));
+  MOE_CU(moe::launch_align_sort(p, grid, stream));
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// grouped FFN
+// ---------------------------------------------------------------------------
+struct FfnShape {
+  int T, H, I, E, k, bm, fp8, tn;
+  long long P, NB, N;
+};
+
+int pick_tn(const FfnShape& s, int hint) {
+  if (hint) return hint;
+  const double avg = (double)s.N / s.E;  // slots per expert
+  long long need = (long long)((avg * 1.25 + s.bm - 1) / s.bm) * s.bm;
+  if (need < s.bm) need = s.bm;
+  int tn = 16;
+  while (tn < need && tn < 256) tn <<= 1;
+  return tn;
+}
+
+moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, int hint, FfnShape* s) {
+  if (!align_args_ok(T, k, E, bm) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (k > 32 || k > E) return MOE_ERR_INVALID_ARG;
+  if (wdtype != MOE_BF16 && wdtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (hint != 0 && hint != 16 && hint != 32 && hint != 64 && hint != 128 && hint != 256)
+    return MOE_ERR_INVALID_ARG;
+  if (H % 128 || I % 128) return MOE_ERR_UNSUPPORTED;
+  s->T = T; s->H = H; s->I = I; s->E = E; s->k = k; s->bm = bm;
+  s->fp8 = wdtype == MOE_FP8_E4M3;
+  s->N = (long long)T * k;
+  s->P = s->N + (long long)E * (bm - 1);
+  s->NB = (s->P + bm - 1) / bm;
+  s->tn = pick_tn(*s, hint);
+  if ((long long)s->P * (s->H > s->I ? s->H : s->I) >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct FfnWs {
+  size_t plan, A, sA, h, hq, sH, total;
+};
+
+FfnWs ffn_ws_layout(const FfnShape& s) {
+  Carver c;
+  FfnWs w;
+  w.plan = c.take((size_t)moe::plan_ints(s.E) * 4);
+  w.A = c.take((size_t)s.P * s.H * (s.fp8 ? 1 : 2));
+  w.sA = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
+  w.h = c.take((size_t)s.P * s.I * 2);
+  w.hq = c.take(s.fp8 ? (size_t)s.P * s.I : 0);
+  w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
+  w.total = c.off;
+  return w;
+}
+
+moe_status_t gemm_fail(int r, const char* what) {
+  if (r == -1) {
+    g_last_cuda_error = std::string(what) + ": cuTensorMapEncodeTiled failed";
+    return MOE_ERR_CUDA;
+  }
+  return cuda_fail((cudaError_t)r, what);
+}
+
+// Runs plan -> gather(+quant) -> gate/up GEMM -> (requant) -> down GEMM.
+moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
+                     const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
+                     const float* topk_w, float* out, bool fused, uint8_t* ws, int32_t* status,
+                     cudaStream_t stream) {
+  const FfnWs L = ffn_ws_layout(s);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
+  void* A = ws + L.A;
+  float* sA = reinterpret_cast<float*>(ws + L.sA);
+  void* h = ws + L.h;
+  void* hq = ws + L.hq;
+  float* sH = reinterpret_cast<float*>(ws + L.sH);
+  const int P = (int)s.P, N = (int)s.N;
+
+  MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, s.H / 128, plan, status, stream));
+  if (s.fp8) MOE_CU(moe::launch_quant_rows(x, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
+  else MOE_CU(moe::launch_permute_bf16(x, sorted, num_post, P, N, s.k, s.H, A, stream));
+
+  moe::GemmLaunch g1 = {};
+  g1.w = w13;
+  g1.w_rows = (long long)s.E * 2 * s.I;
+  g1.x = A;
+  g1.x_rows = s.P;
+  g1.p.gateup = 1;
+  g1.p.fp8 = s.fp8;
+  g1.p.K = s.H;
+  g1.p.n_out = s.I;
+  g1.p.tn = s.tn;
+  g1.p.E = s.E;
+  g1.p.n_slots = N;
+  g1.p.k = s.k;
+  g1.p.plan = plan;
+  g1.p.sorted = sorted;
+  g1.p.a_scale = sA;
+  g1.p.w_scale = w13s;
+  g1.p.out = h;
+  g1.p.status = status;
+  g1.p.timeout_ns = moe::kDefaultTimeoutNs;
+  int r = moe::launch_grouped_gemm(g1, stream);
+  if (r) return gemm_fail(r, "gate/up GEMM");
+
+  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, nullptr, num_post, P, N, s.k, s.I, hq, sH, stream));
+
+  moe::GemmLaunch g2 = {};
+  g2.w = w2;
+  g2.w_rows = (long long)s.E * s.H;
+  g2.x = s.fp8 ? hq : h;
+  g2.x_rows = s.P;
+  g2.p.gateup = 0;
+  g2.p.fp8 = s.fp8;
+  g2.p.K = s.I;
+  g2.p.n_out = s.H;
+  g2.p.tn = s.tn;
+  g2.p.E = s.E;
+  g2.p.n_slots = N;
+  g2.p.k = s.k;
+  g2.p.plan = plan;
+  g2.p.sorted = sorted;
+  g2.p.a_scale = sH;
+  g2.p.w_scale = w2s;
+  g2.p.topk_w = topk_w;
+  g2.p.out = out;
+  g2.p.fused = fused ? 1 : 0;
+  g2.p.status = status;
+  g2.p.timeout_ns = moe::kDefaultTimeoutNs;
+  r = moe::launch_grouped_gemm(g2, stream);
+  if (r) return gemm_fail(r, "down GEMM");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+int moe_version(void) { return 100; }
+
+moe_status_t moe_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* topk_ids,
+                           float* topk_w, void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_topk_gate(logits, bias, T, E, k, topk_ids, topk_w, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status_t moe_align_sort_sizes(int T, int k, int E, int block_size, size_t* P, size_t* NB, size_t* ws_bytes) {
+  if (!align_args_ok(T, k, E, block_size)) return MOE_ERR_INVALID_ARG;
+  const long long p = (long long)T * k + (long long)E * (block_size - 1);
+  if (P) *P = (size_t)p;
+  if (NB) *NB = (size_t)((p + block_size - 1) / block_size);
+  if (ws_bytes) *ws_bytes = align_ws_bytes(E);
+  return MOE_OK;
+}
+
+moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int k, int E, int block_size, int32_t* sorted_ids,
+                            int32_t* expert_ids, int32_t* num_post, void* ws, size_t ws_bytes,
+                            int32_t* dev_status, void* stream) {
+  if (!align_args_ok(T, k, E, block_size)) return MOE_ERR_INVALID_ARG;
+  if (!sorted_ids || !expert_ids || !num_post || !ws || (T > 0 && !topk_ids)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < align_ws_bytes(E)) return MOE_ERR_WORKSPACE;
+  moe_status_t st = check_device();
+  if (st) return st;
+  return run_align(topk_ids, T, k, E, block_size, sorted_ids, expert_ids, num_post, ws, dev_status,
+                   (cudaStream_t)stream);
+}
+
+moe_status_t moe_ffn_workspace(const moe_ffn_args* a, size_t* ws_bytes) {
+  if (!a || !ws_bytes) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  if (st) return st;
+  *ws_bytes = ffn_ws_layout(s).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_grouped_ffn(const moe_ffn_args* a, float* y, void* ws, size_t ws_bytes, int32_t* dev_status,
+                             void* stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  if (st) return st;
+  if (s.N == 0) return MOE_OK;
+  if (!a->x || !a->w13 || !a->w2 || !a->sorted_ids || !a->expert_ids || !a->num_post || !y || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (s.fp8 && (!a->w13_scale || !a->w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->x) || !aligned16(a->w13) || !aligned16(a->w2) || !aligned16(y) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ffn_ws_layout(s).total) return MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st) return st;
+  return run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, a->sorted_ids, a->expert_ids, a->num_post,
+                 nullptr, y, false, static_cast<uint8_t*>(ws), dev_status, (cudaStream_t)stream);
+}
+
+moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int H, void* out, int out_dtype,
+                         void* stream) {
+  if (T < 0 || k < 1 || H < 1 || H % 4) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_BF16 && out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !topk_w || !out || !aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_combine(y, topk_w, T, k, H, out, out_dtype == MOE_BF16, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+namespace {
+struct FwdWs {
+  size_t ids, w, sorted, eids, npost, align, ffn, out32, total;
+};
+FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
+  Carver c;
+  FwdWs w;
+  w.ids = c.take((size_t)s.N * 4);
+  w.w = c.take((size_t)s.N * 4);
+  w.sorted = c.take((size_t)s.P * 4);
+  w.eids = c.take((size_t)s.NB * 4);
+  w.npost = c.take(4);
+  w.align = c.take(align_ws_bytes(s.E));
+  w.ffn = c.take(ffn_ws_layout(s).total);
+  w.out32 = c.take(out_dtype == MOE_BF16 ? (size_t)s.T * s.H * 4 : 0);
+  w.total = c.off;
+  return w;
+}
+}  // namespace
+
+moe_status_t moe_forward_workspace(const moe_forward_args* a, size_t* ws_bytes) {
+  if (!a || !ws_bytes) return MOE_ERR_INVALID_ARG;
+  if (a->out_dtype != MOE_BF16 && a->out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  if (st) return st;
+  *ws_bytes = fwd_ws_layout(s, a->out_dtype).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
+                         void* stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  if (a->out_dtype != MOE_BF16 && a->out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  if (st) return st;
+  if (s.T == 0) return MOE_OK;
+  if (!a->x || !a->logits || !a->w13 || !a->w2 || !a->out || !ws) return MOE_ERR_INVALID_ARG;
+  if (s.fp8 && (!a->w13_scale || !a->w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->x) || !aligned16(a->w13) || !aligned16(a->w2) || !aligned16(a->out) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  const FwdWs L = fwd_ws_layout(s, a->out_dtype);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* ids = a->topk_ids ? a->topk_ids : reinterpret_cast<int32_t*>(w + L.ids);
+  float* tw = a->topk_w ? a->topk_w : reinterpret_cast<float*>(w + L.w);
+  int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
+  int32_t* eids = reinterpret_cast<int32_t*>(w + L.eids);
+  int32_t* npost = reinterpret_cast<int32_t*>(w + L.npost);
+  MOE_CU(moe::launch_topk_gate(a->logits, a->bias, s.T, s.E, s.k, ids, tw, cs));
+  st = run_align(ids, s.T, s.k, s.E, s.bm, sorted, eids, npost, w + L.align, dev_status, cs);
+  if (st) return st;
+  float* out32 = a->out_dtype == MOE_F32 ? static_cast<float*>(a->out) : reinterpret_cast<float*>(w + L.out32);
+  MOE_CU(cudaMemsetAsync(out32, 0, (size_t)s.T * s.H * sizeof(float), cs));
+  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, tw, out32, true,
+               w + L.ffn, dev_status, cs);
+  if (st) return st;
+  if (a->out_dtype == MOE_BF16) MOE_CU(moe::launch_cast_bf16(out32, a->out, (long long)s.T * s.H, cs));
+  return MOE_OK;
+}
+
+moe_status_t moe_test_wait_timeout(void* ws, int32_t* dev_status, long long timeout_ns, void* stream) {
+  if (!ws || !dev_status || timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  MOE_CU(cudaMemsetAsync(ws, 0, sizeof(int), cs));
+  MOE_CU(moe::launch_wait_timeout(static_cast<int*>(ws), dev_status, timeout_ns, cs));
+  return MOE_OK;
+}
+
+}  // extern "C"

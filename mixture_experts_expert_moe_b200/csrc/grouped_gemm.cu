@@ -1,0 +1,461 @@
+// Grouped expert GEMMs of the MoE FFN on sm_100a: tcgen05 MMA with TMEM
+// accumulators, operands staged by TMA into 128-byte-swizzled shared memory.
+//
+// What it computes (MoE Align & Sort article, opening definition and
+// "AITER": each expert's FFN weights multiplied with a block of the tokens
+// routed to it; aiter issue 1248: g1u1 SiLU, per-token FP8; GC-MoE: fused
+// SwiGLU and requantisation):
+//   gate/up : h[r, n] = bf16( silu(G) * U ),  G = Wg[e][n] . A[r],  U = Wu[e][n] . A[r]
+//   down    : y[slot(r), n] = Wd[e][n] . h[r]   (or out[t] += w_slot * y, fused)
+// for every sorted row r of expert e; FP8 operands are rescaled by the
+// per-row activation scale and the per-channel weight scale after the fp32
+// accumulation.
+//
+// Design (B200-first, not the pages' MI300 assembly tiles):
+//   * operand swap (as the GC-MoE abstract describes for Blackwell decode):
+//     128 weight rows fill the MMA M dimension and the expert's tokens are N
+//     (16..256).  An expert's weight tile is streamed once for up to 256 of
+//     its tokens, so weight traffic does not grow with the block size (the
+//     lesson of the aiter issue's I/O table).
+//   * persistent CTAs, one per SM, walk a device-built tile list ordered
+//     expert -> weight tile -> token group, so CTAs that run at the same
+//     time share weight tiles through L2 when an expert has several groups.
+//   * warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread)
+//     and owns the TMEM allocation, warps 2..5 drain TMEM (tcgen05.ld) and
+//     run the epilogue.  An S-stage shared-memory ring (full/empty
+//     mbarriers) decouples TMA from MMA; two TMEM accumulator buffers
+//     decouple MMA from the epilogue when they fit in 512 columns.
+//   * every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
+//     drains its copies and MMAs, frees TMEM and returns.
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kGemmThreads = 192;
+constexpr int kWRows = 128;      // weight rows per tile = MMA M
+constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
+constexpr int kWTileBytes = kWRows * kStageK;
+
+// Plan layout (int32), written by plan_kernel from the align&sort outputs.
+//   [0] tiles of the gate/up GEMM   [1] tiles of the down GEMM   [2] tn
+//   seg_start[E] @4      first sorted row of each expert
+//   seg_rows[E]  @4+E    padded rows of each expert
+//   groups[E]    @4+2E   token groups of <= tn rows
+//   pref_gu[E+1] @4+3E   exclusive prefix of gate/up tiles per expert
+//   pref_dn[E+1] @5+4E   exclusive prefix of down tiles per expert
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ expert_ids,
+                                                    const int32_t* __restrict__ num_post, int P, int E, int bm,
+                                                    int tn, int nw_gu, int nw_dn, int32_t* __restrict__ plan,
+                                                    int32_t* status) {
+  extern __shared__ int sm[];
+  int* s_first = sm;        // first block of expert
+  int* s_nblk = sm + E;     // blocks of expert
+  int* s_pg = sm + 2 * E;   // gate/up tiles -> prefix
+  int* s_pd = sm + 3 * E;   // down tiles -> prefix
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    s_first[e] = 0;
+    s_nblk[e] = 0;
+  }
+  __syncthreads();
+  int np = *num_post;
+  if (np < 0 || np > P || np % bm != 0) {
+    if (tid == 0) dev_flag(status, MOE_DEV_BAD_PLAN);
+    np = 0;
+  }
+  const int nb = np / bm;
+  for (int b = tid; b < nb; b += blockDim.x) {
+    const int e = expert_ids[b];
+    if (e < 0 || e >= E) {
+      dev_flag(status, MOE_DEV_BAD_PLAN);
+      continue;
+    }
+    atomicAdd(&s_nblk[e], 1);
+    if (b == 0 || expert_ids[b - 1] != e) s_first[e] = b;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int rows = s_nblk[e] * bm;
+    const int g = (rows + tn - 1) / tn;
+    plan[4 + e] = s_first[e] * bm;
+    plan[4 + E + e] = rows;
+    plan[4 + 2 * E + e] = g;
+    s_pg[e] = g * nw_gu;
+    s_pd[e] = g * nw_dn;
+  }
+  __syncthreads();
+  if (tid == 0) {  // E <= 1024: a serial scan is a few microseconds at most
+    int a = 0, b = 0;
+    for (int e = 0; e < E; ++e) {
+      plan[4 + 3 * E + e] = a;
+      plan[5 + 4 * E + e] = b;
+      a += s_pg[e];
+      b += s_pd[e];
+    }
+    plan[4 + 4 * E] = a;
+    plan[5 + 5 * E] = b;
+    plan[0] = a;
+    plan[1] = b;
+    plan[2] = tn;
+    plan[3] = np;
+  }
+}
+
+cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
+                        int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 4 * E * sizeof(int), s>>>(expert_ids, num_post, P, E, bm, tn, nw_gu, nw_dn, plan,
+                                                   status);
+  return cudaGetLastError();
+}
+
+
+struct TileInfo {
+  int e, wt, r0, nrows;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_pref, const int* s_start, const int* s_rows,
+                                                const int* s_groups, int E, int tn) {
+  int lo = 0, hi = E - 1;  // last expert whose tile range starts at or before t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_pref[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.e = lo;
+  const int local = t - s_pref[lo];
+  const int G = s_groups[lo];
+  ti.wt = local / G;
+  const int g = local - ti.wt * G;
+  ti.r0 = s_start[lo] + g * tn;
+  ti.nrows = min(tn, s_rows[lo] - g * tn);
+  return ti;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, long long timeout_ns,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int E = p.E;
+  const int w_bytes = p.gateup ? 2 * kWTileBytes : kWTileBytes;
+  const int stage_bytes = w_bytes + p.tn * kStageK;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + p.stages;
+  uint64_t* acc_full = bars + 2 * p.stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
+  int* s_start = s_abort + 3;   // keep 16-byte alignment of the arrays below
+  int* s_rows = s_start + E;
+  int* s_groups = s_rows + E;
+  int* s_pref = s_groups + E;   // E + 1
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, p.tmem_cols);
+    tmem_relinquish();
+  }
+  const int pref_off = p.gateup ? 4 + 3 * E : 5 + 4 * E;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) {
+    s_start[i] = p.plan[4 + i];
+    s_rows[i] = p.plan[4 + E + i];
+    s_groups[i] = p.plan[4 + 2 * E + i];
+  }
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_pref[i] = p.plan[pref_off + i];
+  const int n_tiles = p.plan[p.gateup ? 0 : 1];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  const int nk = p.K * (p.fp8 ? 1 : 2) / kStageK;   // stages per tile
+  const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
+  const int cols_per_acc = p.gateup ? 2 * p.tn : p.tn;
+  volatile int* abort_flag = s_abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long armed = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+        const int wrow = p.gateup ? ti.e * 2 * p.n_out + ti.wt * kWRows : ti.e * p.n_out + ti.wt * kWRows;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = smem + (size_t)stage * stage_bytes;
+          mbar_arrive_expect_tx(&full[stage], stage_bytes);
+          const int kc = kb * k_elems;
+          tma_load_2d(sb, &tm_w, &full[stage], kc, wrow, pol_w);
+          if (p.gateup) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, wrow + p.n_out, pol_w);
+          tma_load_2d(sb + w_bytes, &tm_x, &full[stage], kc, ti.r0, pol_x);
+          ++armed;
+          if (++stage == p.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA exits
+        for (int s = 0; s < p.stages; ++s) {
+          if (armed > s) {
+            const uint32_t par = s < stage ? phase : phase ^ 1;
+            const unsigned long long t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], par) && (long long)(globaltimer_ns() - t0) < 100000000LL) {
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      const uint32_t fmt = p.fp8 ? 0u : 1u;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+        const int acc = it % p.n_acc;
+        const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
+        if (!wait_or_abort(&acc_empty[acc], acc_phase ^ 1, p.timeout_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * cols_per_acc);
+        const uint32_t d1 = d0 + (uint32_t)p.tn;
+        const int n_mma = ((ti.nrows + 15) / 16) * 16;
+        const uint32_t idesc = umma_idesc(kWRows, n_mma, fmt);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, p.timeout_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t w0 = smem_u32(smem + (size_t)stage * stage_bytes);
+          const uint32_t xa = w0 + (uint32_t)w_bytes;
+#pragma unroll
+          for (int kk = 0; kk < kStageK / 32; ++kk) {
+            const uint64_t bdesc = umma_desc_sw128(xa + kk * 32);
+            const uint32_t accum = (kb | kk) != 0;
+            if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
+            else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
+            if (p.gateup) {
+              const uint32_t w1 = w0 + kWTileBytes;
+              if (p.fp8) mma_e4m3(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
+              else mma_bf16(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
+            }
+          }
+          issued = true;
+          tc_commit(&empty[stage]);
+          if (++stage == p.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+      }
+      if (!ok && issued) {
+        // wait for the MMAs in flight before TMEM is freed
+        tc_commit(drain);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < 100000000LL) {
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int m = 32 * q + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      const int acc = it % p.n_acc;
+      const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
+      if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * cols_per_acc);
+      const int n = ti.wt * kWRows + m;
+      if (p.gateup) {
+        float sg = 1.f, su = 1.f;
+        if (p.fp8) {
+          sg = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n);
+          su = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n);
+        }
+        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+        for (int c = 0; c < ti.nrows; c += 16) {
+          float g[16], u[16];
+          tmem_ld16(tb + c, g);
+          tmem_ld16(tb + p.tn + c, u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = c + i;
+            if (j < ti.nrows) {
+              const int row = ti.r0 + j;
+              float gv = g[i], uv = u[i];
+              if (p.fp8) {
+                const float sa = __ldg(p.a_scale + row);
+                gv = gv * sa * sg;
+                uv = uv * sa * su;
+              }
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
+            }
+          }
+        }
+      } else {
+        const float sw = p.fp8 ? __ldg(p.w_scale + (long long)ti.e * p.n_out + n) : 1.f;
+        float* o = reinterpret_cast<float*>(p.out);
+        for (int c = 0; c < ti.nrows; c += 16) {
+          float v[16];
+          tmem_ld16(tb + c, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = c + i;
+            if (j < ti.nrows) {
+              const int row = ti.r0 + j;
+              const int slot = __ldg(p.sorted + row);
+              if (slot < p.n_slots) {
+                float val = v[i];
+                if (p.fp8) val = val * __ldg(p.a_scale + row) * sw;
+                if (p.fused) {
+                  atomicAdd(o + (long long)(slot / p.k) * p.n_out + n, __ldg(p.topk_w + slot) * val);
+                } else {
+                  o[(long long)slot * p.n_out + n] = val;
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) dev_flag(p.status, MOE_DEV_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D K-major tensor [rows, K] with a box of (128 bytes of K) x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, long long rows, long long K, int elem_bytes,
+                     int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K * elem_bytes)};
+  cuuint32_t box[2] = {(cuuint32_t)(kStageK / elem_bytes), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+
+size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
+  const int stage_bytes = (gateup ? 2 : 1) * kWTileBytes + tn * kStageK;
+  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5) * 8 + 16 + (size_t)(4 * E + 1) * 4;
+}
+
+int gemm_pick_stages(int gateup, int tn, int E) {
+  int s = 8;
+  while (s > 2 && gemm_smem_bytes(gateup, tn, s, E) > 225 * 1024) --s;
+  return s;
+}
+
+int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream) {
+  GemmParams& p = L.p;
+  const int eb = p.fp8 ? 1 : 2;
+  CUtensorMap tw, tx;
+  if (!make_map(&tw, L.w, L.w_rows, p.K, eb, kWRows)) return -1;
+  if (!make_map(&tx, L.x, L.x_rows, p.K, eb, p.tn)) return -1;
+  p.stages = gemm_pick_stages(p.gateup, p.tn, p.E);
+  const int cols = p.gateup ? 2 * p.tn : p.tn;
+  p.n_acc = 2 * cols <= 512 ? 2 : 1;
+  int need = p.n_acc * cols, alloc = 32;
+  while (alloc < need) alloc <<= 1;
+  p.tmem_cols = alloc;
+  const size_t smem = gemm_smem_bytes(p.gateup, p.tn, p.stages, p.E);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return (int)e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  grouped_gemm_kernel<<<sms, kGemmThreads, smem, stream>>>(tw, tx, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace moe

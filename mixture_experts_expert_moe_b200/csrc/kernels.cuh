@@ -1,0 +1,82 @@
+// Kernel parameter blocks and launchers shared by the host API (api.cu).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+struct AlignParams {
+  const int32_t* ids;
+  int N;            // T*k flat slots
+  int E;
+  int bm;
+  int chunk;        // slots per CTA, a multiple of 32 * kAlignWarps
+  int32_t* sorted;
+  int32_t* expert_ids;
+  int32_t* num_post;
+  int32_t* hist;    // [gridDim.x][E]
+  int* barrier;     // zeroed before launch
+  int32_t* status;
+  long long timeout_ns;
+  int expected;     // arrivals to wait for (gridDim.x; larger only in the timeout test)
+};
+
+size_t align_smem_bytes(int E);
+cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream);
+int align_max_ctas(int E, int* err_out);
+cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout_ns, cudaStream_t stream);
+
+cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* ids,
+                             float* w, cudaStream_t s);
+cudaError_t launch_permute_bf16(const void* x, const int32_t* sorted, const int32_t* num_post, int P, int N,
+                                int k, int H, void* A, cudaStream_t s);
+cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, const int32_t* num_post, int P, int N,
+                              int k, int C, void* q, float* scale, cudaStream_t s);
+cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
+                           cudaStream_t s);
+cudaError_t launch_cast_bf16(const float* a, void* out, long long n, cudaStream_t s);
+
+// Plan layout (int32), written by the plan kernel from the align&sort outputs:
+//   [0] gate/up tiles  [1] down tiles  [2] tokens per tile  [3] padded rows
+//   seg_start[E] @4, seg_rows[E] @4+E, groups[E] @4+2E,
+//   pref_gu[E+1] @4+3E, pref_dn[E+1] @5+4E
+__host__ __device__ inline int plan_ints(int E) { return 6 + 5 * E; }
+cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
+                        int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s);
+
+struct GemmParams {
+  int gateup;          // 1: gate/up with SiLU*mul epilogue, 0: down projection
+  int fp8;             // E4M3 operands (kind::f8f6f4) instead of bf16 (kind::f16)
+  int K;               // reduction length (elements)
+  int n_out;           // output features per expert: I (gate/up) or H (down)
+  int tn;              // token tile (MMA N), multiple of 16, <= 256
+  int stages;
+  int n_acc;           // TMEM accumulator buffers
+  int tmem_cols;       // allocated TMEM columns (power of two)
+  int E;
+  int n_slots;         // T*k
+  int k;
+  const int32_t* plan;
+  const int32_t* sorted;
+  const float* a_scale;  // [P] per sorted row (FP8)
+  const float* w_scale;  // per weight row (FP8)
+  const float* topk_w;   // [T*k] (down, fused)
+  void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] or out f32 [T, n_out]
+  int fused;             // down: atomically add w*y into out[t]
+  int32_t* status;
+  long long timeout_ns;
+};
+
+struct GemmLaunch {
+  const void* w;        // [E * w_rows_per_expert, K]
+  long long w_rows;     // total weight rows
+  const void* x;        // [P, K]
+  long long x_rows;     // P
+  GemmParams p;
+};
+
+size_t gemm_smem_bytes(int gateup, int tn, int stages, int E);
+int gemm_pick_stages(int gateup, int tn, int E);
+// returns 0 on success, -1 if a tensor map could not be encoded, else a cudaError_t
+int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,88 @@
+"""The C-ABI library loads and exports every entry point that
+include/moe_b200.h declares; host-side argument checks and size queries
+(no device work: these calls return before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_expert_moe_b200 as m
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe_b200.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = m.load_library()
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(m.EXPORTED) == names
+
+
+def test_status_strings_and_version():
+    lib = m.load_library()
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
+    assert lib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
+    assert lib.moe_version() == 100
+
+
+def test_align_sizes():
+    assert m.align_sort_sizes(16384, 8, 256, 64) == (131072 + 256 * 63, -(-(131072 + 256 * 63) // 64),
+                                                     256 + 1024 * 256 * 4)
+    assert m.align_sort_sizes(0, 8, 256, 64)[0] == 256 * 63
+    lib = m.load_library()
+    P = ctypes.c_size_t()
+    assert lib.moe_align_sort_sizes(4, 2, 0, 16, ctypes.byref(P), None, None) == 1
+    assert lib.moe_align_sort_sizes(4, 2, 1025, 16, ctypes.byref(P), None, None) == 1
+    assert lib.moe_align_sort_sizes(4, 0, 8, 16, ctypes.byref(P), None, None) == 1
+    assert lib.moe_align_sort_sizes(-1, 2, 8, 16, ctypes.byref(P), None, None) == 1
+
+
+@pytest.mark.parametrize("bad", [dict(E=0), dict(k=0), dict(k=9), dict(T=-1), dict(E=1025)])
+def test_gate_rejects_bad_sizes(bad):
+    lib = m.load_library()
+    a = dict(T=4, E=8, k=2)
+    a.update(bad)
+    assert lib.moe_topk_gate(None, None, a["T"], a["E"], a["k"], None, None, None) == 1
+
+
+def _ffn(**kw):
+    a = dict(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, tile_tokens=0)
+    a.update(kw)
+    return m.FfnArgs(**a)
+
+
+def test_ffn_workspace_and_validation():
+    lib = m.load_library()
+    n = ctypes.c_size_t()
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn()), ctypes.byref(n)) == 0 and n.value > 0
+    n8 = ctypes.c_size_t()
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=1)), ctypes.byref(n8)) == 0
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(H=200)), ctypes.byref(n)) == 2     # unsupported
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(I=96)), ctypes.byref(n)) == 2
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=2)), ctypes.byref(n)) == 1
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(tile_tokens=48)), ctypes.byref(n)) == 1
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(k=9)), ctypes.byref(n)) == 1
+    # missing pointers are rejected before any launch
+    assert lib.moe_grouped_ffn(ctypes.byref(_ffn()), None, None, 0, None, None) == 1
+
+
+def test_forward_workspace_and_validation():
+    lib = m.load_library()
+    a = m.ForwardArgs(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, out_dtype=0)
+    n = ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)) == 0
+    a.out_dtype = 1
+    assert lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)) == 1
+    a.out_dtype = 2
+    assert lib.moe_forward(ctypes.byref(a), None, 0, None, None) == 1
+    assert lib.moe_combine(None, None, 4, 2, 6, None, 0, None) == 1    # H % 4
+    assert lib.moe_combine(None, None, 4, 2, 8, None, 5, None) == 1    # dtype
