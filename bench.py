@@ -1,0 +1,504 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one full layer forward through the C ABI (``moe_forward``): top-k
+gating, align & sort, gather, gate/up GEMM with SiLU*mul, down GEMM with the
+fused weighted combine, bf16 cast.  The headline workload is the
+DeepSeek-V3-shaped prefill layer (T=2048 tokens, hidden 7168, inter 2048,
+256 experts, top-8, block 64, bf16, router logits ~ N(0,1)).  Its expert
+weights (22.5 GB) are far larger than L2, so no flush is needed between
+steps.  Extra objects in the line report the a8w8 variant, the
+Mixtral-shaped prefill, the a8w8 decode sweep and align & sort alone
+(16384 tokens, top-8 of 256, Zipf s=1, block 64; L2 flushed between calls).
+
+Multi-GPU: the layer does not shard here, so N GPUs run N independent
+replicas ("scaling": "weak"); the time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_inputs import ALIGN_CONFIG, CONFIGS, align_ids, make_layer  # noqa: E402
+from mixture_experts_expert_moe_b200.roofline import (  # noqa: E402
+    align_bytes, expert_weight_bytes, layer_bytes, moe_flops)
+
+METRIC = "MoE layer tokens/s & TFLOPS vs roofline (bf16/fp8); align&sort µs, GB/s"
+PRIMARY = CONFIGS["deepseek"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_name(cfg, dtype):
+    return (f"{cfg.name}_{dtype}: T={cfg.T} H={cfg.H} I={cfg.I} E={cfg.E} k={cfg.k} bm={cfg.bm}"
+            f"{' +bias' if cfg.bias else ''}")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device.index or 0)
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != 7:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        smax = max(r[1] for r in rows)
+        load = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in load])), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def build_layer(m, cfg, dev, out_dtype=torch.bfloat16):
+    d = make_layer(cfg, device=dev)
+    if cfg.a8w8:
+        layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype)
+    else:
+        layer = m.MoELayer(d["w13"], d["w2"], cfg.k, cfg.bm, out_dtype=out_dtype)
+    return d, layer
+
+
+def touched_experts(layer, d):
+    ids = torch.empty(d["x"].shape[0], layer.k, dtype=torch.int32, device=d["x"].device)
+    layer(d["x"], d["logits"], d["bias"], topk_ids=ids)
+    torch.cuda.synchronize()
+    return int(torch.unique(ids).numel()), ids
+
+
+def kernels_per_step(cfg, out_dtype):
+    n = 7 if out_dtype == torch.bfloat16 else 6   # gate, align, plan, gather, gate/up, down, cast
+    return n + (1 if cfg.a8w8 else 0)             # + requant
+
+
+def time_layer(m, cfg, layer, d, steps, warmup, stage_times=True):
+    dev = d["x"].device
+    out = torch.empty(cfg.T, cfg.H, dtype=layer.out_dtype, device=dev)
+    for _ in range(warmup):
+        layer(d["x"], d["logits"], d["bias"], out=out)
+    nst = len(m.STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(steps)] if stage_times else None
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        layer(d["x"], d["logits"], d["bias"], out=out, stage_events=evs[i] if evs else None)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    st = None
+    if evs:
+        st = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, name in enumerate(m.STAGES)}
+    return ms, st
+
+
+def time_e2e(cfg, layer, d, steps, warmup):
+    """Same layer through the C ABI with host buffers: pinned x and logits
+    copied in and the output copied out inside the timed region."""
+    dev = d["x"].device
+    xh = d["x"].cpu().pin_memory()
+    lh = d["logits"].cpu().pin_memory()
+    oh = torch.empty(cfg.T, cfg.H, dtype=layer.out_dtype).pin_memory()
+    xd, ld = torch.empty_like(d["x"]), torch.empty_like(d["logits"])
+    out = torch.empty(cfg.T, cfg.H, dtype=layer.out_dtype, device=dev)
+
+    def step():
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        layer(xd, ld, d["bias"], out=out)
+        oh.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    h2d = xh.numel() * xh.element_size() + lh.numel() * lh.element_size()
+    d2h = oh.numel() * oh.element_size()
+    return ms, h2d, d2h
+
+
+def gateup_bytes(cfg, touched):
+    eb = 1 if cfg.a8w8 else 2
+    pairs = cfg.T * cfg.k
+    w = touched * (2 * cfg.I * cfg.H * eb + (8 * cfg.I if cfg.a8w8 else 0))
+    return w + pairs * cfg.H * eb + pairs * cfg.I * 2
+
+
+def down_bytes(cfg, touched):
+    eb = 1 if cfg.a8w8 else 2
+    pairs = cfg.T * cfg.k
+    w = touched * (cfg.H * cfg.I * eb + (4 * cfg.H if cfg.a8w8 else 0))
+    return w + pairs * cfg.I * eb + cfg.T * cfg.H * 4
+
+
+def traffic_for(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        tab = json.load(f)
+    ent = tab.get(f"{kernel}|{workload}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
+    return ent["bytes_per_launch"] if h == ent.get("source_sha") else None
+
+
+def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False):
+    d, layer = build_layer(m, cfg, dev)
+    touched, _ = touched_experts(layer, d)
+    ms, st = time_layer(m, cfg, layer, d, steps, warmup)
+    step_ms = ms / steps
+    pairs = cfg.T * cfg.k
+    fl = moe_flops(pairs, cfg.H, cfg.I)
+    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k, touched, cfg.I, cfg.a8w8)
+    tf_peak = pk["bf16_tflops_sustained"] * (2.0 if cfg.a8w8 else 1.0)
+    t_roof = max(fl / (tf_peak * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
+    rep = {"workload": workload_name(cfg, dtype_name), "tokens_per_s": cfg.T / (step_ms * 1e-3),
+           "ms_per_step": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12, "touched_experts": touched,
+           "layer_roofline_ms": t_roof, "layer_roofline_frac": t_roof / step_ms,
+           "layer_bound": "tensor" if fl / (tf_peak * 1e12) > by / (pk["hbm_gbs"] * 1e9) else "hbm",
+           "stages_ms": st}
+    # dominant kernel
+    dom = max(st, key=st.get)
+    kb = {"gateup": gateup_bytes(cfg, touched), "down": down_bytes(cfg, touched)}
+    kfl = {"gateup": 4.0 * pairs * cfg.H * cfg.I, "down": 2.0 * pairs * cfg.H * cfg.I}
+    roof = None
+    if dom in kb:
+        t = st[dom] * 1e-3
+        hbm_t = kb[dom] / (pk["hbm_gbs"] * 1e9)
+        ten_t = kfl[dom] / (tf_peak * 1e12)
+        if ten_t > hbm_t:
+            roof = {"kernel": f"grouped_gemm_kernel ({dom})", "bound": "tensor", "achieved": kfl[dom] / t / 1e12,
+                    "peak": tf_peak, "unit": "TFLOP/s"}
+        else:
+            roof = {"kernel": f"grouped_gemm_kernel ({dom})", "bound": "hbm", "achieved": kb[dom] / t / 1e9,
+                    "peak": pk["hbm_gbs"], "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = traffic_for(f"grouped_gemm_{dom}", rep["workload"])
+        roof["algorithmic_bytes"] = kb[dom]
+        roof["launch_ms"] = st[dom]
+    rep["dominant"] = roof
+    e2e = None
+    if primary:
+        ems, h2d, d2h = time_e2e(cfg, layer, d, max(10, steps // 2), 3)
+        e2e = {"value": cfg.T * max(10, steps // 2) / (ems * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del layer, d
+    torch.cuda.empty_cache()
+    return rep, e2e, ms
+
+
+def align_report(m, dev, pk, T, iters=100):
+    E, k, bm = ALIGN_CONFIG["E"], ALIGN_CONFIG["k"], ALIGN_CONFIG["bm"]
+    ids = torch.from_numpy(align_ids(T, E, k, seed=ALIGN_CONFIG["seed"], dist="zipf",
+                                     zipf_s=ALIGN_CONFIG["zipf_s"])).to(dev)
+    P, NB, wsb = m.align_sort_sizes(T, k, E, bm)
+    out = (torch.empty(P, dtype=torch.int32, device=dev), torch.empty(NB, dtype=torch.int32, device=dev),
+           torch.empty(1, dtype=torch.int32, device=dev))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(5):
+        m.align_sort(ids, E, bm, ws=ws, out=out)
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.align_sort(ids, E, bm, ws=ws, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    us = float(np.median(ts)) * 1e3
+    n = int(out[2].item())
+    by = align_bytes(T * k, n, bm)
+    gbs = by / (us * 1e-6) / 1e9
+    return {"workload": f"align_sort: T={T} E={E} k={k} bm={bm} zipf s=1, L2 flushed", "us": us,
+            "gb_per_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "algorithmic_bytes": by}
+
+
+def run_ours(args):
+    import mixture_experts_expert_moe_b200 as m
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    m.load_library()
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    pk, pk_src = peaks()
+    cfg = PRIMARY
+    d, layer = build_layer(m, cfg, dev)
+    touched, _ = touched_experts(layer, d)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        layer(d["x"], d["logits"], d["bias"], out=out)
+    nst = len(m.STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        layer(d["x"], d["logits"], d["bias"], out=out, stage_events=evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    stages = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, name in enumerate(m.STAGES)}
+    step_ms = ms / args.steps
+    pairs = cfg.T * cfg.k
+    fl = moe_flops(pairs, cfg.H, cfg.I)
+    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k, touched, cfg.I, False)
+    t_roof = max(fl / (pk["bf16_tflops_sustained"] * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
+    dom = max(stages, key=stages.get)
+    kbytes = {"gateup": gateup_bytes(cfg, touched), "down": down_bytes(cfg, touched)}.get(dom)
+    roof = None
+    if kbytes is not None:
+        ach = kbytes / (stages[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"],
+                "traffic": traffic_for(f"grouped_gemm_{dom}", workload_name(cfg, "bf16")),
+                "kernel": f"grouped_gemm_kernel ({dom} projection)", "launch_ms": stages[dom],
+                "algorithmic_bytes": kbytes, "peak_source": f"{pk_src} hbm_gbs (copy)"}
+    ems, h2d, d2h = time_e2e(cfg, layer, d, max(10, args.steps // 2), 3)
+    e2e = {"value": world * cfg.T * max(10, args.steps // 2) / (ems * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del layer, d
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if rank == 0 and not args.quick:
+        extra["a8w8"], _, _ = layer_report(m, cfg.with_(a8w8=True), 50, 5, dev, pk, "a8w8")
+        extra["mixtral"], _, _ = layer_report(m, CONFIGS["mixtral"], 20, 3, dev, pk, "bf16")
+        extra["decode_a8w8"] = []
+        for T in (1, 16, 64, 256):
+            r, _, _ = layer_report(m, CONFIGS["decode"].with_(T=T), 100, 5, dev, pk, "a8w8")
+            extra["decode_a8w8"].append(r)
+        extra["align_sort"] = align_report(m, dev, pk, ALIGN_CONFIG["T"])
+        extra["align_sort_large"] = align_report(m, dev, pk, 1 << 22, iters=20)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(cfg)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": world * cfg.T * args.steps / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) random-init expert weights)",
+        "config": {"workload": workload_name(cfg, "bf16"), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (22.5 GB of expert weights streamed per step)",
+                   "touched_experts": touched},
+        "tflops": fl / (step_ms * 1e-3) / 1e12,
+        "layer_roofline": {"ms": t_roof, "frac": t_roof / step_ms, "bound": "hbm",
+                           "bytes": by, "flops": fl, "peak_source": pk_src},
+        "stages_ms": stages,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": kernels_per_step(cfg, torch.bfloat16) * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    line.update(extra)
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+class _HostExperts:
+    """Expert weights of the experts a sample touches, copied to the host once
+    (float32, or bf16 converted on access); the oracle converts each expert it
+    uses to float64 itself."""
+
+    def __init__(self, t, needed, as_f32):
+        self.shape = tuple(t.shape)
+        self.as_f32 = as_f32
+        self.host = {int(e): (t[int(e)].float().cpu().numpy() if as_f32 else t[int(e)].cpu()) for e in needed}
+
+    def __getitem__(self, e):
+        w = self.host[int(e)]
+        return w if self.as_f32 else w.float().numpy()
+
+
+def _oracle_inputs(cfg, n_tokens, as_f32, seed=0):
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if torch.cuda.is_available() else "cpu"
+    d = make_layer(cfg, device=dev)
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(cfg.T, size=n_tokens, replace=False))
+    x = d["x"][torch.from_numpy(toks).to(d["x"].device)].float().cpu().numpy()
+    logits = d["logits"][torch.from_numpy(toks).to(d["x"].device)].cpu().numpy()
+    # experts the sampled tokens route to (for the host copy only; the oracle routes itself)
+    need = torch.topk(d["logits"][torch.from_numpy(toks).to(d["x"].device)], cfg.k, dim=1).indices.unique().cpu()
+    w13 = _HostExperts(d["w13"], need, as_f32)
+    w2 = _HostExperts(d["w2"], need, as_f32)
+    del d
+    if torch.cuda.is_available():
+        torch.cuda.empty_cache()
+    return x, logits, w13, w2
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, n_tokens=6):
+    import oracle
+    x, logits, w13, w2 = _oracle_inputs(cfg, n_tokens, as_f32=False)
+    t = time.perf_counter()
+    oracle.moe_forward(x, logits, cfg.k, w13, w2)
+    dt = time.perf_counter() - t
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"a batch of {n_tokens} seeded tokens of {workload_name(cfg, 'bf16')} through the "
+                      f"whole layer (float64 numpy; bf16 weights converted per expert), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = PRIMARY
+    n_tokens = 1
+    x, logits, w13, w2 = _oracle_inputs(cfg, n_tokens, as_f32=True)
+    for _ in range(args.warmup):
+        oracle.moe_forward(x, logits, cfg.k, w13, w2)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_forward(x, logits, cfg.k, w13, w2)
+    dt = time.perf_counter() - t
+    v = n_tokens * args.steps / dt
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    sample = (f"a batch of {n_tokens} seeded token per step of {workload_name(cfg, 'bf16')} through the "
+              f"whole layer (float64 numpy on the host; the token's experts' weights held as float32)")
+    print(json.dumps({
+        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(cfg, "bf16"), "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline workload only")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        args.steps = 3 if args.steps is None else args.steps
+        args.warmup = 1 if args.warmup is None else args.warmup
+        run_reference(args)
+    else:
+        args.steps = 100 if args.steps is None else args.steps
+        args.warmup = 5 if args.warmup is None else max(3, args.warmup)
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -198,7 +198,22 @@ typedef struct {
   int32_t* topk_ids;          /* nullable: routing also written here [T,k] */
   float* topk_w;              /* nullable [T,k]                           */
   int tile_tokens;            /* as in moe_ffn_args                       */
+  void** stage_events;        /* nullable: MOE_NUM_STAGES + 1 cudaEvent_t
+                                 handles; event 0 is recorded before the first
+                                 stage and event i+1 after stage i, on
+                                 `stream` (for per-stage timing)           */
 } moe_forward_args;
+
+/* Stages of moe_forward, in launch order (stage_events indices). */
+#define MOE_STAGE_GATE 0      /* top-k gating                              */
+#define MOE_STAGE_ALIGN 1     /* align & sort                              */
+#define MOE_STAGE_PLAN 2      /* tile list for the grouped GEMMs           */
+#define MOE_STAGE_GATHER 3    /* token rows to sorted order (+FP8 quant)   */
+#define MOE_STAGE_GATEUP 4    /* gate/up GEMM with SiLU*mul                */
+#define MOE_STAGE_REQUANT 5   /* FP8 requantisation of h (empty for bf16)  */
+#define MOE_STAGE_DOWN 6      /* down GEMM with the fused weighted combine */
+#define MOE_STAGE_CAST 7      /* fp32 -> bf16 output (empty for f32 out)   */
+#define MOE_NUM_STAGES 8
 
 MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);
 MOE_API moe_status_t moe_forward(const moe_forward_args* args, void* ws, size_t ws_bytes,

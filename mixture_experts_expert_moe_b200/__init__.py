@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_BF16, MOE_FP8_E4M3, MOE_F32 = 0, 1, 2
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN = 0x1, 0x2, 0x4
+STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "cast"]
 
 EXPORTED = [
     "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
@@ -40,7 +41,7 @@ class ForwardArgs(ctypes.Structure):
     _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i),
                 ("wdtype", _i), ("out_dtype", _i), ("x", _vp), ("logits", _vp), ("bias", _vp),
                 ("w13", _vp), ("w13_scale", _vp), ("w2", _vp), ("w2_scale", _vp), ("out", _vp),
-                ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i)]
+                ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i), ("stage_events", _vp)]
 
 
 _LIB = None
@@ -217,7 +218,7 @@ class MoELayer:
         self.I = twoI // 2
         self._ws = None
 
-    def _args(self, x, logits, bias, out, ids, w):
+    def _args(self, x, logits, bias, out, ids, w, events=None):
         T = x.shape[0]
         return ForwardArgs(
             T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
@@ -226,7 +227,8 @@ class MoELayer:
             w13=self.w13.data_ptr(), w13_scale=None if self.w13_scale is None else self.w13_scale.data_ptr(),
             w2=self.w2.data_ptr(), w2_scale=None if self.w2_scale is None else self.w2_scale.data_ptr(),
             out=out.data_ptr(), topk_ids=None if ids is None else ids.data_ptr(),
-            topk_w=None if w is None else w.data_ptr(), tile_tokens=self.tile_tokens)
+            topk_w=None if w is None else w.data_ptr(), tile_tokens=self.tile_tokens,
+            stage_events=None if events is None else ctypes.cast(events, ctypes.c_void_p))
 
     def workspace_bytes(self, T):
         lib = load_library()
@@ -238,7 +240,10 @@ class MoELayer:
         _check(lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)), "moe_forward_workspace")
         return n.value
 
-    def __call__(self, x, logits, bias=None, out=None, topk_ids=None, topk_w=None, dev_status=None):
+    def __call__(self, x, logits, bias=None, out=None, topk_ids=None, topk_w=None, dev_status=None,
+                 stage_events=None):
+        """Run the layer.  ``stage_events``: optional list of len(STAGES)+1
+        torch.cuda.Event objects recorded at the stage boundaries."""
         lib = load_library()
         T = x.shape[0]
         if out is None:
@@ -246,7 +251,14 @@ class MoELayer:
         need = self.workspace_bytes(T)
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.empty(need, dtype=torch.uint8, device=x.device)
-        a = self._args(x, logits, bias, out, topk_ids, topk_w)
+        evs = None
+        if stage_events is not None:
+            assert len(stage_events) == len(STAGES) + 1
+            for e in stage_events:
+                if e.cuda_event == 0:     # created lazily by torch
+                    e.record()
+            evs = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+        a = self._args(x, logits, bias, out, topk_ids, topk_w, evs)
         _check(lib.moe_forward(ctypes.byref(a), _ptr(self._ws), self._ws.numel(),
                                _dev_status(dev_status, x.device), _stream(x.device)), "moe_forward")
         return out

@@ -35,6 +35,10 @@ struct Carver {
   }
 };
 
+inline cudaError_t record(void** ev, int i, cudaStream_t s) {
+  return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 moe_status_t check_device() {
@@ -160,7 +164,7 @@ moe_status_t gemm_fail(int r, const char* what) {
 moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
                      const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
                      const float* topk_w, float* out, bool fused, uint8_t* ws, int32_t* status,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, void** ev = nullptr) {
   const FfnWs L = ffn_ws_layout(s);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
@@ -171,8 +175,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   const int P = (int)s.P, N = (int)s.N;
 
   MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, s.H / 128, plan, status, stream));
+  MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
   if (s.fp8) MOE_CU(moe::launch_quant_rows(x, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
   else MOE_CU(moe::launch_permute_bf16(x, sorted, num_post, P, N, s.k, s.H, A, stream));
+  MOE_CU(record(ev, MOE_STAGE_GATHER + 1, stream));
 
   moe::GemmLaunch g1 = {};
   g1.w = w13;
@@ -196,8 +202,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
+  MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
 
   if (s.fp8) MOE_CU(moe::launch_quant_rows(h, nullptr, num_post, P, N, s.k, s.I, hq, sH, stream));
+  MOE_CU(record(ev, MOE_STAGE_REQUANT + 1, stream));
 
   moe::GemmLaunch g2 = {};
   g2.w = w2;
@@ -223,6 +231,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
+  MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
   return MOE_OK;
 }
 
@@ -371,15 +380,21 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
   int32_t* eids = reinterpret_cast<int32_t*>(w + L.eids);
   int32_t* npost = reinterpret_cast<int32_t*>(w + L.npost);
+  void** ev = a->stage_events;
+  float* out32 = a->out_dtype == MOE_F32 ? static_cast<float*>(a->out) : reinterpret_cast<float*>(w + L.out32);
+  MOE_CU(record(ev, 0, cs));
   MOE_CU(moe::launch_topk_gate(a->logits, a->bias, s.T, s.E, s.k, ids, tw, cs));
+  MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   st = run_align(ids, s.T, s.k, s.E, s.bm, sorted, eids, npost, w + L.align, dev_status, cs);
   if (st) return st;
-  float* out32 = a->out_dtype == MOE_F32 ? static_cast<float*>(a->out) : reinterpret_cast<float*>(w + L.out32);
+  // zeroing the fused-combine accumulator belongs to the align stage's tail
   MOE_CU(cudaMemsetAsync(out32, 0, (size_t)s.T * s.H * sizeof(float), cs));
+  MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
   st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, tw, out32, true,
-               w + L.ffn, dev_status, cs);
+               w + L.ffn, dev_status, cs, ev);
   if (st) return st;
   if (a->out_dtype == MOE_BF16) MOE_CU(moe::launch_cast_bf16(out32, a->out, (long long)s.T * s.H, cs));
+  MOE_CU(record(ev, MOE_STAGE_CAST + 1, cs));
   return MOE_OK;
 }
 
