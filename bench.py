@@ -481,6 +481,29 @@ def run_reference(args):
     }))
 
 
+def run_only(args):
+    import mixture_experts_expert_moe_b200 as m
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pk, _ = peaks()
+    steps = 20 if args.steps is None else args.steps
+    warmup = 3 if args.warmup is None else max(3, args.warmup)
+    parts = args.only.split("_")
+    if parts[0] == "align":
+        print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
+        return
+    cfg = CONFIGS[parts[0]].with_(a8w8=parts[1] == "a8w8")
+    for p in parts[2:]:
+        if p.startswith("bm"):
+            cfg = cfg.with_(bm=int(p[2:]))
+        elif p.startswith("T"):
+            cfg = cfg.with_(T=int(p[1:]))
+        elif p == "bias":
+            cfg = cfg.with_(bias=True)
+    rep, _, _ = layer_report(m, cfg, steps, warmup, dev, pk, parts[1])
+    print(json.dumps(rep))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -489,7 +512,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--only", default=None,
+                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>] "
+                         "(configs: tiny, p5, deepseek, mixtral, decode) or align_<T>")
     args = ap.parse_args()
+    if args.only:
+        run_only(args)
+        return
     if args.impl == "reference":
         args.steps = 3 if args.steps is None else args.steps
         args.warmup = 1 if args.warmup is None else args.warmup

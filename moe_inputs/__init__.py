@@ -65,6 +65,8 @@ CONFIGS = {
     # DeepSeek-V3-shaped prefill (uniform routing); a8w8 / bias / bm variants
     "deepseek": MoEConfig("deepseek", T=2048, H=7168, I=2048, E=256, k=8, bm=64,
                           seed=SEED_BASE + 3),
+    # the aiter a8w8 issue's shape: 32 local experts, ~64 tokens each
+    "p5": MoEConfig("p5", T=256, H=7168, I=2048, E=32, k=8, bm=64, seed=SEED_BASE + 5),
     # decode sweep, FP8 a8w8 (T in 1, 16, 64, 256)
     "decode": MoEConfig("decode", T=64, H=7168, I=2048, E=256, k=8, bm=16,
                         a8w8=True, seed=SEED_BASE + 4),
