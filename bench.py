@@ -5,7 +5,7 @@
 
 A step is one full layer forward through the C ABI (``moe_forward``): top-k
 gating, align & sort, gather, gate/up GEMM with SiLU*mul, down GEMM with the
-fused weighted combine, bf16 cast.  The headline workload is the
+per-slot expert outputs, weighted combine.  The headline workload is the
 DeepSeek-V3-shaped prefill layer (T=2048 tokens, hidden 7168, inter 2048,
 256 experts, top-8, block 64, bf16, router logits ~ N(0,1)).  Its expert
 weights (22.5 GB) are far larger than L2, so no flush is needed between
@@ -136,7 +136,7 @@ def touched_experts(layer, d):
 
 
 def kernels_per_step(cfg, out_dtype):
-    n = 7 if out_dtype == torch.bfloat16 else 6   # gate, align, plan, gather, gate/up, down, cast
+    n = 7                                         # gate, align, plan, gather, gate/up, down, combine
     return n + (1 if cfg.a8w8 else 0)             # + requant
 
 
@@ -159,6 +159,27 @@ def time_layer(m, cfg, layer, d, steps, warmup, stage_times=True):
     if evs:
         st = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, name in enumerate(m.STAGES)}
     return ms, st
+
+
+def time_graph(m, cfg, layer, d, steps, warmup):
+    """Replays of one captured forward (CUDA graph); None if capture fails."""
+    out = torch.empty(cfg.T, cfg.H, dtype=layer.out_dtype, device=d["x"].device)
+    try:
+        g, _ = m.capture_graph(layer, d["x"], d["logits"], d["bias"], out=out)
+    except Exception as exc:  # report eager numbers only
+        sys.stderr.write(f"graph capture failed: {exc}\n")
+        return None
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    del g
+    return t0.elapsed_time(t1)
 
 
 def time_e2e(cfg, layer, d, steps, warmup):
@@ -203,7 +224,7 @@ def down_bytes(cfg, touched):
     eb = 1 if cfg.a8w8 else 2
     pairs = cfg.T * cfg.k
     w = touched * (cfg.H * cfg.I * eb + (4 * cfg.H if cfg.a8w8 else 0))
-    return w + pairs * cfg.I * eb + cfg.T * cfg.H * 4
+    return w + pairs * cfg.I * eb + pairs * cfg.H * 4     # + y, one fp32 row per slot
 
 
 def traffic_for(kernel, workload):
@@ -225,7 +246,9 @@ def traffic_for(kernel, workload):
 def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False):
     d, layer = build_layer(m, cfg, dev)
     touched, _ = touched_experts(layer, d)
-    ms, st = time_layer(m, cfg, layer, d, steps, warmup)
+    ms_eager, st = time_layer(m, cfg, layer, d, steps, warmup)
+    ms_graph = time_graph(m, cfg, layer, d, steps, warmup)
+    ms = ms_graph if ms_graph is not None else ms_eager
     step_ms = ms / steps
     pairs = cfg.T * cfg.k
     fl = moe_flops(pairs, cfg.H, cfg.I)
@@ -236,7 +259,8 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False):
            "ms_per_step": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12, "touched_experts": touched,
            "layer_roofline_ms": t_roof, "layer_roofline_frac": t_roof / step_ms,
            "layer_bound": "tensor" if fl / (tf_peak * 1e12) > by / (pk["hbm_gbs"] * 1e9) else "hbm",
-           "stages_ms": st}
+           "stages_ms": st, "launch": "cuda_graph" if ms_graph is not None else "eager",
+           "eager_ms_per_step": ms_eager / steps}
     # dominant kernel
     dom = max(st, key=st.get)
     kb = {"gateup": gateup_bytes(cfg, touched), "down": down_bytes(cfg, touched)}
@@ -278,20 +302,34 @@ def align_report(m, dev, pk, T, iters=100):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(5):
         m.align_sort(ids, E, bm, ws=ws, out=out)
+    torch.cuda.synchronize()
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            m.align_sort(ids, E, bm, ws=ws, out=out)
+    except Exception as exc:
+        sys.stderr.write(f"align graph capture failed: {exc}\n")
+        graph = None
     ts = []
-    for _ in range(iters):
+    for it in range(iters + 3):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        m.align_sort(ids, E, bm, ws=ws, out=out)
+        if graph is not None:
+            graph.replay()
+        else:
+            m.align_sort(ids, E, bm, ws=ws, out=out)
         b.record()
         torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
+        if it >= 3:
+            ts.append(a.elapsed_time(b))
     us = float(np.median(ts)) * 1e3
     n = int(out[2].item())
     by = align_bytes(T * k, n, bm)
     gbs = by / (us * 1e-6) / 1e9
-    return {"workload": f"align_sort: T={T} E={E} k={k} bm={bm} zipf s=1, L2 flushed", "us": us,
+    return {"workload": f"align_sort: T={T} E={E} k={k} bm={bm} zipf s=1, L2 flushed",
+            "launch": "cuda_graph" if graph is not None else "eager", "us": us,
             "gb_per_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "algorithmic_bytes": by}
 
 
@@ -311,11 +349,22 @@ def run_ours(args):
     cfg = PRIMARY
     d, layer = build_layer(m, cfg, dev)
     touched, _ = touched_experts(layer, d)
+    ms_eager, stages = time_layer(m, cfg, layer, d, args.steps, args.warmup)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    graph = None
+    try:
+        graph, _ = m.capture_graph(layer, d["x"], d["logits"], d["bias"], out=out)
+    except Exception as exc:
+        sys.stderr.write(f"graph capture failed, timing eager launches: {exc}\n")
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            layer(d["x"], d["logits"], d["bias"], out=out)
+
     for _ in range(args.warmup):
-        layer(d["x"], d["logits"], d["bias"], out=out)
-    nst = len(m.STAGES) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+        step()
     clocks = ClockSampler(dev)
     clocks.start()
     time.sleep(0.3)
@@ -324,8 +373,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
-    for i in range(args.steps):
-        layer(d["x"], d["logits"], d["bias"], out=out, stage_events=evs[i])
+    for _ in range(args.steps):
+        step()
     t1.record()
     torch.cuda.synchronize()
     if world > 1:
@@ -336,7 +385,8 @@ def run_ours(args):
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    stages = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, name in enumerate(m.STAGES)}
+    used_graph = graph is not None
+    del graph
     step_ms = ms / args.steps
     pairs = cfg.T * cfg.k
     fl = moe_flops(pairs, cfg.H, cfg.I)
@@ -383,7 +433,9 @@ def run_ours(args):
         "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) random-init expert weights)",
         "config": {"workload": workload_name(cfg, "bf16"), "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (22.5 GB of expert weights streamed per step)",
-                   "touched_experts": touched},
+                   "touched_experts": touched,
+                   "launch": "cuda_graph replay of one moe_forward" if used_graph else "eager moe_forward"},
+        "eager_ms_per_step": ms_eager / args.steps,
         "tflops": fl / (step_ms * 1e-3) / 1e12,
         "layer_roofline": {"ms": t_roof, "frac": t_roof / step_ms, "bound": "hbm",
                            "bytes": by, "flops": fl, "peak_source": pk_src},

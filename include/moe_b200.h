@@ -179,9 +179,10 @@ MOE_API moe_status_t moe_combine(const float* y, const float* topk_w, int T, int
                          void* out, int out_dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
- * moe_forward -- gate, align & sort, grouped FFN and combine in one call.
- * The combine is fused into the down projection (fp32 atomic accumulation,
- * so the summation order over the k choices is not fixed).
+ * moe_forward -- gate, align & sort, grouped FFN and combine in one call:
+ * the same arithmetic as moe_topk_gate, moe_align_sort, moe_grouped_ffn and
+ * moe_combine in sequence (per-slot expert outputs kept in the workspace,
+ * combined in fp32 in ascending j, so the result is deterministic).
  * ------------------------------------------------------------------------- */
 typedef struct {
   int T, H, I, E, k, block_size;
@@ -211,8 +212,8 @@ typedef struct {
 #define MOE_STAGE_GATHER 3    /* token rows to sorted order (+FP8 quant)   */
 #define MOE_STAGE_GATEUP 4    /* gate/up GEMM with SiLU*mul                */
 #define MOE_STAGE_REQUANT 5   /* FP8 requantisation of h (empty for bf16)  */
-#define MOE_STAGE_DOWN 6      /* down GEMM with the fused weighted combine */
-#define MOE_STAGE_CAST 7      /* fp32 -> bf16 output (empty for f32 out)   */
+#define MOE_STAGE_DOWN 6      /* down GEMM, one fp32 row per slot          */
+#define MOE_STAGE_COMBINE 7   /* top-k weighted combine into out           */
 #define MOE_NUM_STAGES 8
 
 MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);

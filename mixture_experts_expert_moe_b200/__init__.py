@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_BF16, MOE_FP8_E4M3, MOE_F32 = 0, 1, 2
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN = 0x1, 0x2, 0x4
-STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "cast"]
+STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "combine"]
 
 EXPORTED = [
     "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
@@ -262,6 +262,20 @@ class MoELayer:
         _check(lib.moe_forward(ctypes.byref(a), _ptr(self._ws), self._ws.numel(),
                                _dev_status(dev_status, x.device), _stream(x.device)), "moe_forward")
         return out
+
+
+def capture_graph(layer, x, logits, bias=None, out=None):
+    """Capture one ``layer`` forward on these fixed buffers into a CUDA graph.
+
+    Returns (graph, out); ``graph.replay()`` reruns the whole forward (the
+    same kernels the C ABI launches) without host launch overhead.
+    """
+    out = layer(x, logits, bias, out=out)      # sizes the workspace outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer(x, logits, bias, out=out)
+    return g, out
 
 
 def run_wait_timeout_check(timeout_ns: int, device="cuda"):

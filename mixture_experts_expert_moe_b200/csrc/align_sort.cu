@@ -9,16 +9,16 @@
 //       one leader updates the row (no atomics, and the order is fixed).
 //   (C) cumulative sums: the warp rows are scanned into per-warp exclusive
 //       prefixes (the article's "unaligned local cumsum"), the CTA totals go
-//       to a global matrix hist[cta][expert] (the "merge" through a
+//       to a global matrix hist[expert][cta] (the "merge" through a
 //       preallocated HBM buffer), and after the single grid-wide wait every
-//       CTA reads the matrix column-wise to get its own prefix and the
-//       expert totals, pads the totals to the block size and scans them (the
-//       "aligned global cumsum").
+//       CTA reads each expert's row with coalesced warp loads to get its own
+//       prefix and the expert totals, pads the totals to the block size and
+//       scans them (the "aligned global cumsum").
 //   (P) parallel placement: each warp re-reads its sub-chunk and writes every
 //       slot to  offset[e] + (slots of e in earlier CTAs) + (in earlier warps)
 //       + (earlier in this warp), which is the stable counting-sort position.
-//       Block expert ids and sentinel padding are written by the CTA that
-//       owns the block.
+//       Block expert ids and the sentinel padding (only in an expert's last
+//       block) are written by the CTA that owns the block.
 // Unlike the article's design there is no second kernel and no single-block
 // alignment step: every CTA redoes the small E-wide scan itself, which costs
 // less than another launch or grid-wide wait.
@@ -26,9 +26,9 @@
 
 namespace moe {
 
-constexpr int kAlignThreads = 512;
+constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
-
+constexpr int kSub = 8;  // 32-slot sub-steps a warp loads before it processes them
 
 // Grid-wide wait with a time limit; returns false if it ran out.
 __device__ bool grid_wait(int* counter, int expected, long long timeout_ns) {
@@ -40,7 +40,7 @@ __device__ bool grid_wait(int* counter, int expected, long long timeout_ns) {
     int ok = 1;
     unsigned long long t0 = globaltimer_ns();
     while (ld_acquire_gpu(counter) < expected) {
-      __nanosleep(100);
+      __nanosleep(64);
       if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
         ok = 0;
         break;
@@ -94,9 +94,31 @@ __device__ int block_exclusive_scan(int* a, int n) {
   return s_total;
 }
 
-__global__ void __launch_bounds__(kAlignThreads) align_sort_kernel(AlignParams p) {
+// Loads kSub sub-steps (32 consecutive slots each) of a warp's sub-chunk;
+// ids outside [0, E) and slots past the end become -1.
+__device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, long long end, int lane, int E,
+                                          int (&key)[kSub]) {
+  bool bad = false;
+#pragma unroll
+  for (int q = 0; q < kSub; ++q) {
+    const long long i = base + q * 32 + lane;
+    int v = -1;
+    if (i < end) {
+      v = __ldg(ids + i);
+      if (v < 0 || v >= E) {
+        bad = true;
+        v = -1;
+      }
+    }
+    key[q] = v;
+  }
+  return bad;
+}
+
+__global__ void __launch_bounds__(kAlignThreads, 1) align_sort_kernel(AlignParams p) {
   extern __shared__ int smem[];
   const int E = p.E;
+  const int G = gridDim.x;
   int* wcnt = smem;                       // [kAlignWarps][E] per-warp counts, then prefixes
   int* s_off = wcnt + kAlignWarps * E;    // [E] padded segment offsets
   int* s_base = s_off + E;                // [E] this CTA's first position per expert
@@ -114,44 +136,29 @@ __global__ void __launch_bounds__(kAlignThreads) align_sort_kernel(AlignParams p
   const long long w_end = min((long long)p.N, w_begin + wsub);
   int* my = wcnt + warp * E;
 
-  // ---- (D) count ----------------------------------------------------------
+  // ---- (D) count: each warp into its own row -------------------------------
   bool bad = false;
-  for (long long base = w_begin; base < w_end; base += 128) {
-    int key[4];
+  for (long long base = w_begin; base < w_end; base += 32 * kSub) {
+    int key[kSub];
+    bad |= load_keys(p.ids, base, w_end, lane, E, key);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      long long i = base + q * 32 + lane;
-      int v = -1;
-      if (i < w_end) {
-        v = __ldg(p.ids + i);
-        if (v < 0 || v >= E) {
-          bad = true;
-          v = -1;
-        }
-      }
-      key[q] = v;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      unsigned peers = __match_any_sync(0xffffffffu, key[q]);
-      if (key[q] >= 0 && (peers & lanemask_lt()) == 0) my[key[q]] += __popc(peers);
-      __syncwarp();
-    }
+    for (int q = 0; q < kSub; ++q)
+      if (key[q] >= 0) atomicAdd(&my[key[q]], 1);
   }
   if (bad) s_bad = 1;
   __syncthreads();
   if (tid == 0 && s_bad) dev_flag(p.status, MOE_DEV_BAD_EXPERT_ID);
 
-  // per-warp exclusive prefixes inside the CTA; CTA totals to the matrix
+  // per-warp exclusive prefixes inside the CTA; CTA totals to column b of hist[e][b]
   for (int e = tid; e < E; e += blockDim.x) {
     int run = 0;
-#pragma unroll 4
+#pragma unroll 8
     for (int w = 0; w < kAlignWarps; ++w) {
-      int c = wcnt[w * E + e];
+      const int c = wcnt[w * E + e];
       wcnt[w * E + e] = run;
       run += c;
     }
-    p.hist[(long long)blockIdx.x * E + e] = run;
+    p.hist[(long long)e * G + blockIdx.x] = run;
   }
 
   if (!grid_wait(p.barrier, p.expected, p.timeout_ns)) {
@@ -159,29 +166,40 @@ __global__ void __launch_bounds__(kAlignThreads) align_sort_kernel(AlignParams p
     return;
   }
 
-  // ---- (C) this CTA's prefix, totals, padded offsets ----------------------
-  const int ncta = gridDim.x;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int pre = 0, tot = 0;
-    int b = 0;
-    for (; b + 8 <= ncta; b += 8) {
-      int c[8];
+  // ---- (C) own prefix and expert totals from row e of hist ------------------
+  // warp w reduces experts w, w+32, ...; lane l reads CTAs l, l+32, ...
+  for (int e0 = warp; e0 < E; e0 += kAlignWarps * 8) {
+    int pre[8], tot[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) c[u] = __ldcg(p.hist + (long long)(b + u) * E + e);
+    for (int u = 0; u < 8; ++u) pre[u] = tot[u] = 0;
+    for (int c = 0; c < G; c += 32) {
+      const int b = c + lane;
+      int v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        pre += (b + u < (int)blockIdx.x) ? c[u] : 0;
-        tot += c[u];
+        const int e = e0 + u * kAlignWarps;
+        v[u] = (e < E && b < G) ? __ldcg(p.hist + (long long)e * G + b) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        pre[u] += b < (int)blockIdx.x ? v[u] : 0;
+        tot[u] += v[u];
       }
     }
-    for (; b < ncta; ++b) {
-      int c = __ldcg(p.hist + (long long)b * E + e);
-      pre += (b < (int)blockIdx.x) ? c : 0;
-      tot += c;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        pre[u] += __shfl_xor_sync(0xffffffffu, pre[u], off);
+        tot[u] += __shfl_xor_sync(0xffffffffu, tot[u], off);
+      }
+      const int e = e0 + u * kAlignWarps;
+      if (lane == 0 && e < E) {
+        s_tot[e] = tot[u];
+        s_base[e] = pre[u];
+        s_off[e] = (tot[u] + p.bm - 1) / p.bm * p.bm;
+      }
     }
-    s_tot[e] = tot;
-    s_base[e] = pre;
-    s_off[e] = (tot + p.bm - 1) / p.bm * p.bm;
   }
   __syncthreads();
   const int total_post = block_exclusive_scan(s_off, E);
@@ -191,41 +209,30 @@ __global__ void __launch_bounds__(kAlignThreads) align_sort_kernel(AlignParams p
 
   // ---- block expert ids and sentinel padding for this CTA's blocks -------
   const int nblk = total_post / p.bm;
-  const int bpc = (nblk + ncta - 1) / ncta;
+  const int bpc = (nblk + G - 1) / G;
   const int j0 = blockIdx.x * bpc;
   const int j1 = min(nblk, j0 + bpc);
-  if (j1 > j0) {
-    const long long npos = (long long)(j1 - j0) * p.bm;
-    for (long long idx = tid; idx < npos; idx += blockDim.x) {
-      const long long pos = (long long)j0 * p.bm + idx;
-      int lo = 0, hi = E - 1;  // last expert whose segment starts at or before pos
-      while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
-      }
-      if (idx % p.bm == 0) p.expert_ids[pos / p.bm] = lo;
-      if (pos >= (long long)s_off[lo] + s_tot[lo]) p.sorted[pos] = p.N;
+  for (int j = j0 + tid; j < j1; j += blockDim.x) {
+    const int pos = j * p.bm;
+    int lo = 0, hi = E - 1;  // last expert whose segment starts at or before pos
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
     }
+    p.expert_ids[j] = lo;
+    const int fill = s_off[lo] + s_tot[lo];  // first padding position of expert lo
+    for (int q = max(fill, pos); q < pos + p.bm; ++q) p.sorted[q] = p.N;
   }
 
   // ---- (P) stable placement ------------------------------------------------
-  for (long long base = w_begin; base < w_end; base += 128) {
-    int key[4];
+  for (long long base = w_begin; base < w_end; base += 32 * kSub) {
+    int key[kSub];
+    load_keys(p.ids, base, w_end, lane, E, key);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      long long i = base + q * 32 + lane;
-      int v = -1;
-      if (i < w_end) {
-        v = __ldg(p.ids + i);
-        if (v < 0 || v >= E) v = -1;
-      }
-      key[q] = v;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kSub; ++q) {
       const int kq = key[q];
-      unsigned peers = __match_any_sync(0xffffffffu, kq);
-      int cnt = kq >= 0 ? my[kq] : 0;
+      const unsigned peers = __match_any_sync(0xffffffffu, kq);
+      const int cnt = kq >= 0 ? my[kq] : 0;
       __syncwarp();
       if (kq >= 0) {
         const unsigned below = peers & lanemask_lt();
@@ -240,9 +247,6 @@ __global__ void __launch_bounds__(kAlignThreads) align_sort_kernel(AlignParams p
 size_t align_smem_bytes(int E) { return (size_t)(kAlignWarps + 3) * E * sizeof(int); }
 
 cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)align_smem_bytes(p.E));
-  if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kAlignThreads);
@@ -256,19 +260,32 @@ cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t strea
   return cudaLaunchKernelEx(&cfg, align_sort_kernel, p);
 }
 
+// Largest cooperative grid: one CTA per SM (the column reads of phase C grow
+// with the grid).  The function attribute and occupancy are set up once per
+// device (they depend only on the device and the kernel).
 int align_max_ctas(int E, int* err_out) {
-  int dev = 0, sms = 0, per_sm = 0;
+  static int cached_sms[64] = {0};
+  static int cached_smem[64] = {0};
+  int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)align_smem_bytes(E));
-  if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, align_sort_kernel, kAlignThreads,
-                                                      align_smem_bytes(E));
   *err_out = (int)e;
   if (e != cudaSuccess) return 0;
-  return sms * (per_sm < 1 ? 0 : 1);  // one CTA per SM: the column reads grow with the grid
+  const int need = (int)align_smem_bytes(1024);
+  if (dev < 64 && cached_sms[dev] > 0 && cached_smem[dev] >= need) return cached_sms[dev];
+  int sms = 0, per_sm = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, align_sort_kernel, kAlignThreads, need);
+  *err_out = (int)e;
+  if (e != cudaSuccess || per_sm < 1) return 0;
+  (void)E;
+  if (dev < 64) {
+    cached_sms[dev] = sms;
+    cached_smem[dev] = need;
+  }
+  return sms;
 }
 
 // Timeout test: the same wait on a counter that can never fill.

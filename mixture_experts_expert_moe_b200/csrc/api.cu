@@ -70,8 +70,8 @@ moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t*
   const int max_ctas = moe::align_max_ctas(E, &err);
   if (err) return cuda_fail((cudaError_t)err, "align occupancy");
   if (max_ctas < 1) return MOE_ERR_UNSUPPORTED;
-  const int per_cta_unit = 32 * 16;  // warps x lanes
-  int grid = (N + kMinSlotsPerCta - 1) / kMinSlotsPerCta;
+  const int per_cta_unit = 32 * 32;  // warps x lanes
+  int grid = (int)(((long long)N + kMinSlotsPerCta - 1) / kMinSlotsPerCta);
   grid = grid < 1 ? 1 : grid;
   grid = grid > max_ctas ? max_ctas : grid;
   grid = grid > kMaxAlignCtas ? kMaxAlignCtas : grid;
@@ -163,8 +163,7 @@ moe_status_t gemm_fail(int r, const char* what) {
 // Runs plan -> gather(+quant) -> gate/up GEMM -> (requant) -> down GEMM.
 moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
                      const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
-                     const float* topk_w, float* out, bool fused, uint8_t* ws, int32_t* status,
-                     cudaStream_t stream, void** ev = nullptr) {
+                     float* y, uint8_t* ws, int32_t* status, cudaStream_t stream, void** ev = nullptr) {
   const FfnWs L = ffn_ws_layout(s);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
@@ -224,9 +223,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.sorted = sorted;
   g2.p.a_scale = sH;
   g2.p.w_scale = w2s;
-  g2.p.topk_w = topk_w;
-  g2.p.out = out;
-  g2.p.fused = fused ? 1 : 0;
+  g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
   r = moe::launch_grouped_gemm(g2, stream);
@@ -312,7 +309,7 @@ moe_status_t moe_grouped_ffn(const moe_ffn_args* a, float* y, void* ws, size_t w
   st = check_device();
   if (st) return st;
   return run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, a->sorted_ids, a->expert_ids, a->num_post,
-                 nullptr, y, false, static_cast<uint8_t*>(ws), dev_status, (cudaStream_t)stream);
+                 y, static_cast<uint8_t*>(ws), dev_status, (cudaStream_t)stream);
 }
 
 moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int H, void* out, int out_dtype,
@@ -329,7 +326,7 @@ moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int 
 
 namespace {
 struct FwdWs {
-  size_t ids, w, sorted, eids, npost, align, ffn, out32, total;
+  size_t ids, w, sorted, eids, npost, align, ffn, y, total;
 };
 FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
   Carver c;
@@ -341,7 +338,8 @@ FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
   w.npost = c.take(4);
   w.align = c.take(align_ws_bytes(s.E));
   w.ffn = c.take(ffn_ws_layout(s).total);
-  w.out32 = c.take(out_dtype == MOE_BF16 ? (size_t)s.T * s.H * 4 : 0);
+  w.y = c.take((size_t)s.N * s.H * 4);
+  (void)out_dtype;
   w.total = c.off;
   return w;
 }
@@ -381,20 +379,18 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   int32_t* eids = reinterpret_cast<int32_t*>(w + L.eids);
   int32_t* npost = reinterpret_cast<int32_t*>(w + L.npost);
   void** ev = a->stage_events;
-  float* out32 = a->out_dtype == MOE_F32 ? static_cast<float*>(a->out) : reinterpret_cast<float*>(w + L.out32);
+  float* y = reinterpret_cast<float*>(w + L.y);
   MOE_CU(record(ev, 0, cs));
   MOE_CU(moe::launch_topk_gate(a->logits, a->bias, s.T, s.E, s.k, ids, tw, cs));
   MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   st = run_align(ids, s.T, s.k, s.E, s.bm, sorted, eids, npost, w + L.align, dev_status, cs);
   if (st) return st;
-  // zeroing the fused-combine accumulator belongs to the align stage's tail
-  MOE_CU(cudaMemsetAsync(out32, 0, (size_t)s.T * s.H * sizeof(float), cs));
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
-  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, tw, out32, true,
-               w + L.ffn, dev_status, cs, ev);
+  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, y, w + L.ffn, dev_status,
+               cs, ev);
   if (st) return st;
-  if (a->out_dtype == MOE_BF16) MOE_CU(moe::launch_cast_bf16(out32, a->out, (long long)s.T * s.H, cs));
-  MOE_CU(record(ev, MOE_STAGE_CAST + 1, cs));
+  MOE_CU(moe::launch_combine(y, tw, s.T, s.k, s.H, a->out, a->out_dtype == MOE_BF16, cs));
+  MOE_CU(record(ev, MOE_STAGE_COMBINE + 1, cs));
   return MOE_OK;
 }
 

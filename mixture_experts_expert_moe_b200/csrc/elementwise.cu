@@ -5,7 +5,6 @@
 //                  requantisation of h between the two GEMMs), optionally
 //                  fused with the gather
 //   combine        top-k weighted sum of the per-slot expert outputs
-//   cast_out       fp32 -> bf16 of the fused-combine accumulator
 #include <cfloat>
 
 #include "kernels.cuh"
@@ -244,29 +243,6 @@ cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, 
   dim3 grid((unsigned)((H / 4 + 255) / 256), (unsigned)T), block(256);
   if (bf16) combine_kernel<true><<<grid, block, 0, s>>>((const float4*)y, w, T, k, H, out);
   else combine_kernel<false><<<grid, block, 0, s>>>((const float4*)y, w, T, k, H, out);
-  return cudaGetLastError();
-}
-
-// fp32 -> bf16, 4 per thread (n % 4 == 0).
-__global__ void __launch_bounds__(256) cast_bf16_kernel(const float4* __restrict__ a, uint2* __restrict__ o,
-                                                        long long n4) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-       i += (long long)gridDim.x * blockDim.x) {
-    const float4 v = __ldg(a + i);
-    __nv_bfloat162 x = __floats2bfloat162_rn(v.x, v.y), y = __floats2bfloat162_rn(v.z, v.w);
-    uint2 r;
-    r.x = *reinterpret_cast<uint32_t*>(&x);
-    r.y = *reinterpret_cast<uint32_t*>(&y);
-    o[i] = r;
-  }
-}
-
-cudaError_t launch_cast_bf16(const float* a, void* out, long long n, cudaStream_t s) {
-  if (n == 0) return cudaSuccess;
-  const long long n4 = n / 4;
-  long long g = (n4 + 255) / 256;
-  if (g > 148 * 16) g = 148 * 16;
-  cast_bf16_kernel<<<(unsigned)g, 256, 0, s>>>((const float4*)a, (uint2*)out, n4);
   return cudaGetLastError();
 }
 

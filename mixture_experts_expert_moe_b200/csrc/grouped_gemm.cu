@@ -6,7 +6,7 @@
 // routed to it; aiter issue 1248: g1u1 SiLU, per-token FP8; GC-MoE: fused
 // SwiGLU and requantisation):
 //   gate/up : h[r, n] = bf16( silu(G) * U ),  G = Wg[e][n] . A[r],  U = Wu[e][n] . A[r]
-//   down    : y[slot(r), n] = Wd[e][n] . h[r]   (or out[t] += w_slot * y, fused)
+//   down    : y[slot(r), n] = Wd[e][n] . h[r]
 // for every sorted row r of expert e; FP8 operands are rescaled by the
 // per-row activation scale and the per-channel weight scale after the fp32
 // accumulation.
@@ -365,11 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (slot < p.n_slots) {
                 float val = v[i];
                 if (p.fp8) val = val * __ldg(p.a_scale + row) * sw;
-                if (p.fused) {
-                  atomicAdd(o + (long long)(slot / p.k) * p.n_out + n, __ldg(p.topk_w + slot) * val);
-                } else {
-                  o[(long long)slot * p.n_out + n] = val;
-                }
+                o[(long long)slot * p.n_out + n] = val;
               }
             }
           }

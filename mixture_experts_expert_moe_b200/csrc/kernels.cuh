@@ -13,7 +13,7 @@ struct AlignParams {
   int32_t* sorted;
   int32_t* expert_ids;
   int32_t* num_post;
-  int32_t* hist;    // [gridDim.x][E]
+  int32_t* hist;    // [E][gridDim.x] per-CTA counts
   int* barrier;     // zeroed before launch
   int32_t* status;
   long long timeout_ns;
@@ -33,7 +33,6 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, const int3
                               int k, int C, void* q, float* scale, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
-cudaError_t launch_cast_bf16(const float* a, void* out, long long n, cudaStream_t s);
 
 // Plan layout (int32), written by the plan kernel from the align&sort outputs:
 //   [0] gate/up tiles  [1] down tiles  [2] tokens per tile  [3] padded rows
@@ -59,9 +58,7 @@ struct GemmParams {
   const int32_t* sorted;
   const float* a_scale;  // [P] per sorted row (FP8)
   const float* w_scale;  // per weight row (FP8)
-  const float* topk_w;   // [T*k] (down, fused)
-  void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] or out f32 [T, n_out]
-  int fused;             // down: atomically add w*y into out[t]
+  void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] (one row per slot)
   int32_t* status;
   long long timeout_ns;
 };
