@@ -173,7 +173,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   float* sH = reinterpret_cast<float*>(ws + L.sH);
   const int P = (int)s.P, N = (int)s.N;
 
-  MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, s.H / 128, plan, status, stream));
+  MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status, stream));
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
   if (s.fp8) MOE_CU(moe::launch_quant_rows(x, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
   else MOE_CU(moe::launch_permute_bf16(x, sorted, num_post, P, N, s.k, s.H, A, stream));

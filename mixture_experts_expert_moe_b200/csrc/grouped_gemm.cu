@@ -148,13 +148,19 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
   }
 }
 
+// Token rows of the tile are loaded in boxes of x_box rows, only as many as
+// the token group has (rounded up to x_box).
+__device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int E = p.E;
-  const int w_bytes = p.gateup ? 2 * kWTileBytes : kWTileBytes;
+  // every tile multiplies two 128-row weight sub-tiles with the same token
+  // tile: gate and up rows (gate/up), or output rows n0 and n0+128 (down)
+  const int w_bytes = 2 * kWTileBytes;
   const int stage_bytes = w_bytes + p.tn * kStageK;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
   uint64_t* full = bars;
@@ -205,7 +211,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int nk = p.K * (p.fp8 ? 1 : 2) / kStageK;   // stages per tile
   const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
-  const int cols_per_acc = p.gateup ? 2 * p.tn : p.tn;
+  const int cols_per_acc = 2 * p.tn;
+  const int xb = x_box_rows(p.tn);
   volatile int* abort_flag = s_abort;
 
   if (warp == 0) {
@@ -219,18 +226,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
-        const int wrow = p.gateup ? ti.e * 2 * p.n_out + ti.wt * kWRows : ti.e * p.n_out + ti.wt * kWRows;
+        int row0, row1;
+        bool has1 = true;
+        if (p.gateup) {
+          row0 = ti.e * 2 * p.n_out + ti.wt * kWRows;
+          row1 = row0 + p.n_out;
+        } else {
+          row0 = ti.e * p.n_out + ti.wt * 2 * kWRows;
+          row1 = row0 + kWRows;
+          has1 = ti.wt * 2 * kWRows + kWRows < p.n_out;
+        }
+        const int nload = (ti.nrows + xb - 1) / xb;
+        const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* sb = smem + (size_t)stage * stage_bytes;
-          mbar_arrive_expect_tx(&full[stage], stage_bytes);
+          mbar_arrive_expect_tx(&full[stage], tx);
           const int kc = kb * k_elems;
-          tma_load_2d(sb, &tm_w, &full[stage], kc, wrow, pol_w);
-          if (p.gateup) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, wrow + p.n_out, pol_w);
-          tma_load_2d(sb + w_bytes, &tm_x, &full[stage], kc, ti.r0, pol_x);
+          tma_load_2d(sb, &tm_w, &full[stage], kc, row0, pol_w);
+          if (has1) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, row1, pol_w);
+          for (int l = 0; l < nload; ++l)
+            tma_load_2d(sb + w_bytes + l * xb * kStageK, &tm_x, &full[stage], kc, ti.r0 + l * xb, pol_x);
           ++armed;
           if (++stage == p.stages) {
             stage = 0;
@@ -261,6 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t fmt = p.fp8 ? 0u : 1u;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+        const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
         const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
         if (!wait_or_abort(&acc_empty[acc], acc_phase ^ 1, p.timeout_ns, abort_flag)) {
@@ -279,6 +299,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after();
           const uint32_t w0 = smem_u32(smem + (size_t)stage * stage_bytes);
+          const uint32_t w1 = w0 + kWTileBytes;
           const uint32_t xa = w0 + (uint32_t)w_bytes;
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
@@ -286,8 +307,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t accum = (kb | kk) != 0;
             if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
-            if (p.gateup) {
-              const uint32_t w1 = w0 + kWTileBytes;
+            if (has1) {
               if (p.fp8) mma_e4m3(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
               else mma_bf16(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
             }
@@ -322,8 +342,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * cols_per_acc);
-      const int n = ti.wt * kWRows + m;
       if (p.gateup) {
+        const int n = ti.wt * kWRows + m;
         float sg = 1.f, su = 1.f;
         if (p.fp8) {
           sg = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n);
@@ -351,11 +371,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        const float sw = p.fp8 ? __ldg(p.w_scale + (long long)ti.e * p.n_out + n) : 1.f;
+        const int n0 = ti.wt * 2 * kWRows + m;
+        const int n1 = n0 + kWRows;
+        const bool has1 = n1 < p.n_out;   // uniform across the warp (n_out % 128 == 0)
+        float sw0 = 1.f, sw1 = 1.f;
+        if (p.fp8) {
+          sw0 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n0);
+          if (has1) sw1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
+        }
         float* o = reinterpret_cast<float*>(p.out);
         for (int c = 0; c < ti.nrows; c += 16) {
-          float v[16];
-          tmem_ld16(tb + c, v);
+          float v0[16], v1[16];
+          tmem_ld16(tb + c, v0);
+          if (has1) tmem_ld16(tb + p.tn + c, v1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int j = c + i;
@@ -363,9 +391,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const int row = ti.r0 + j;
               const int slot = __ldg(p.sorted + row);
               if (slot < p.n_slots) {
-                float val = v[i];
-                if (p.fp8) val = val * __ldg(p.a_scale + row) * sw;
-                o[(long long)slot * p.n_out + n] = val;
+                const float sa = p.fp8 ? __ldg(p.a_scale + row) : 1.f;
+                float* yr = o + (long long)slot * p.n_out;
+                yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
+                if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
               }
             }
           }
@@ -422,7 +451,8 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, long long
 
 
 size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
-  const int stage_bytes = (gateup ? 2 : 1) * kWTileBytes + tn * kStageK;
+  const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
+  (void)gateup;
   return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5) * 8 + 16 + (size_t)(4 * E + 1) * 4;
 }
 
@@ -437,9 +467,9 @@ int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream) {
   const int eb = p.fp8 ? 1 : 2;
   CUtensorMap tw, tx;
   if (!make_map(&tw, L.w, L.w_rows, p.K, eb, kWRows)) return -1;
-  if (!make_map(&tx, L.x, L.x_rows, p.K, eb, p.tn)) return -1;
+  if (!make_map(&tx, L.x, L.x_rows, p.K, eb, p.tn < 32 ? p.tn : 32)) return -1;
   p.stages = gemm_pick_stages(p.gateup, p.tn, p.E);
-  const int cols = p.gateup ? 2 * p.tn : p.tn;
+  const int cols = 2 * p.tn;
   p.n_acc = 2 * cols <= 512 ? 2 : 1;
   int need = p.n_acc * cols, alloc = 32;
   while (alloc < need) alloc <<= 1;
