@@ -228,19 +228,21 @@ def down_bytes(cfg, touched):
 
 
 def traffic_for(kernel, workload):
-    """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """dram bytes per launch from the committed ncu summary table
+    (profiles/traffic.md), if it was taken on the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
-    with open(p) as f:
-        tab = json.load(f)
-    ent = tab.get(f"{kernel}|{workload}")
-    if not ent:
-        return None
-    src = os.path.join(ROOT, ent["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
-    return ent["bytes_per_launch"] if h == ent.get("source_sha") else None
+    for line in open(p):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) < 5 or cells[0] != kernel or cells[1] != workload:
+            continue
+        src = os.path.join(ROOT, cells[3])
+        if not os.path.exists(src):
+            return None
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return int(cells[2]) if h == cells[4] else None
+    return None
 
 
 def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False):
