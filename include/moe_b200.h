@@ -125,6 +125,27 @@ MOE_API moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int k, int E
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_align_sort_noalloc -- moe_align_sort without a caller workspace.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory (code running while another framework's
+ * memory pool is frozen, plain C hosts that only receive pointers, runtimes
+ * that forbid cudaMalloc after start-up).  Inputs, outputs, results and
+ * device-status bits are exactly those of moe_align_sort; only the scratch
+ * differs: a fixed device array inside the library (MOE_NOALLOC_SCRATCH_BYTES,
+ * held by every GPU that loads the library until the process exits).
+ * Limit: E <= MOE_NOALLOC_MAX_EXPERTS, otherwise MOE_ERR_UNSUPPORTED and
+ * nothing is launched.  The first call on a device looks up the array's
+ * device address (make that call before any stream capture).  All calls
+ * share the array: calls that overlap on the GPU race; order them on one
+ * stream.  Allocates nothing.
+ * ------------------------------------------------------------------------- */
+#define MOE_NOALLOC_MAX_EXPERTS 256
+#define MOE_NOALLOC_SCRATCH_BYTES (256 + 256 * 256 * 4)
+MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, int T, int k, int E, int block_size,
+                                            int32_t* sorted_ids, int32_t* expert_ids, int32_t* num_post,
+                                            int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_grouped_ffn -- gated grouped expert FFN over the sorted slots.
  * Passage: MoE Align & Sort article, opening definition (expert FFNs on the
  * chosen tokens computed by a Group GEMM) and "AITER" (the grouped GEMM

@@ -24,6 +24,7 @@ EXPORTED = [
     "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
     "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
     "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
+    "moe_align_sort_noalloc",
 ]
 
 _vp = ctypes.c_void_p
@@ -69,6 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_forward_workspace": (_i, [ctypes.POINTER(ForwardArgs), sz]),
             "moe_forward": (_i, [ctypes.POINTER(ForwardArgs), _vp, ctypes.c_size_t, _vp, _vp]),
             "moe_test_wait_timeout": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
+            "moe_align_sort_noalloc": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
