@@ -136,13 +136,15 @@ moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, in
 }
 
 struct FfnWs {
-  size_t plan, A, sA, h, hq, sH, total;
+  size_t plan, xq, sx, A, sA, h, hq, sH, total;
 };
 
 FfnWs ffn_ws_layout(const FfnShape& s) {
   Carver c;
   FfnWs w;
   w.plan = c.take((size_t)moe::plan_ints(s.E) * 4);
+  w.xq = c.take(s.fp8 ? (size_t)s.T * s.H : 0);
+  w.sx = c.take(s.fp8 ? (size_t)s.T * 4 : 0);
   w.A = c.take((size_t)s.P * s.H * (s.fp8 ? 1 : 2));
   w.sA = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
   w.h = c.take((size_t)s.P * s.I * 2);
@@ -168,6 +170,8 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
   float* sA = reinterpret_cast<float*>(ws + L.sA);
+  void* xq = ws + L.xq;
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
   void* h = ws + L.h;
   void* hq = ws + L.hq;
   float* sH = reinterpret_cast<float*>(ws + L.sH);
@@ -175,8 +179,13 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
 
   MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status, stream));
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
-  if (s.fp8) MOE_CU(moe::launch_quant_rows(x, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
-  else MOE_CU(moe::launch_permute_bf16(x, sorted, num_post, P, N, s.k, s.H, A, stream));
+  if (s.fp8) {
+    // quantise each token once, then gather codes and scales into sorted order
+    MOE_CU(moe::launch_quant_rows(x, nullptr, s.T, s.H, xq, sx, stream));
+    MOE_CU(moe::launch_gather_rows(xq, sx, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
+  } else {
+    MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, P, N, s.k, s.H * 2, A, nullptr, stream));
+  }
   MOE_CU(record(ev, MOE_STAGE_GATHER + 1, stream));
 
   moe::GemmLaunch g1 = {};
@@ -203,7 +212,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
 
-  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, nullptr, num_post, P, N, s.k, s.I, hq, sH, stream));
+  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, num_post, P, s.I, hq, sH, stream));
   MOE_CU(record(ev, MOE_STAGE_REQUANT + 1, stream));
 
   moe::GemmLaunch g2 = {};

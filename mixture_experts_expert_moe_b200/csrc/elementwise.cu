@@ -1,9 +1,9 @@
 // Memory-bound steps of the MoE layer forward on sm_100a:
 //   topk_gate      softmax top-k gating, one warp per token
-//   permute        gather of token rows into sorted (expert-grouped) order
+//   gather_rows    token rows (bf16, or E4M3 codes + scale) into sorted
+//                  (expert-grouped) order
 //   quant_rows     per-row E4M3 quantisation (per-token activations, and the
-//                  requantisation of h between the two GEMMs), optionally
-//                  fused with the gather
+//                  requantisation of h between the two GEMMs)
 //   combine        top-k weighted sum of the per-slot expert outputs
 #include <cfloat>
 
@@ -94,25 +94,41 @@ cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int 
 
 // ---------------------------------------------------------------------------
 // Gather of token rows into sorted order (MoE Align & Sort article,
-// "FasterTransformer": permute before the group GEMM).  Row r of A is the
-// token of slot sorted[r]; padding rows are zero.  Rows >= num_post are not
-// touched.  16-byte vectors; H % 8 == 0.
+// "FasterTransformer": permute before the group GEMM).  Row r of dst is the
+// row of token sorted[r] / k (bf16 activations, or their E4M3 codes with the
+// per-token scale); padding rows are zero (scale 1).  Rows >= num_post are not
+// touched.  One warp per row, 16-byte vectors.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) permute_bf16_kernel(const uint4* __restrict__ x,
-                                                           const int32_t* __restrict__ sorted,
-                                                           const int32_t* __restrict__ num_post, int N, int k,
-                                                           int H, uint4* __restrict__ A) {
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
+                                                          const float* __restrict__ src_scale,
+                                                          const int32_t* __restrict__ sorted,
+                                                          const int32_t* __restrict__ num_post, int N, int k,
+                                                          int vec, uint4* __restrict__ dst,
+                                                          float* __restrict__ dst_scale) {
   const int np = *num_post;
-  const int vec = H / 8;
-  for (int r = blockIdx.x; r < np; r += gridDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < np; r += gridDim.x * wpb) {
     const int slot = __ldg(sorted + r);
-    const uint4* src = slot < N ? x + (long long)(slot / k) * vec : nullptr;
-    uint4* dst = A + (long long)r * vec;
-    for (int c = threadIdx.x; c < vec; c += blockDim.x) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (src) v = __ldg(src + c);
-      dst[c] = v;
+    const long long t = slot < N ? slot / k : -1;
+    const uint4* row = t >= 0 ? src + t * vec : nullptr;
+    uint4* out = dst + (long long)r * vec;
+    int c = lane;
+    for (; c + 96 < vec; c += 128) {   // four independent 16-byte loads in flight per lane
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0, v2 = v0, v3 = v0;
+      if (row) {
+        v0 = __ldg(row + c);
+        v1 = __ldg(row + c + 32);
+        v2 = __ldg(row + c + 64);
+        v3 = __ldg(row + c + 96);
+      }
+      out[c] = v0;
+      out[c + 32] = v1;
+      out[c + 64] = v2;
+      out[c + 96] = v3;
     }
+    for (; c < vec; c += 32) out[c] = row ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
+    if (dst_scale && lane == 0) dst_scale[r] = t >= 0 ? __ldg(src_scale + t) : 1.f;
   }
 }
 
@@ -120,8 +136,8 @@ __global__ void __launch_bounds__(256) permute_bf16_kernel(const uint4* __restri
 // Per-row E4M3 quantisation (aiter issue 1248: per-token FP8 activations;
 // GC-MoE: requantisation between the GEMMs).  s = amax / 448 in fp32 (1 for
 // an all-zero row); code = e4m3_rne_satfinite(v / s) with an IEEE fp32
-// division.  In gather mode row r reads token sorted[r] / k of x (padding
-// rows become zero codes with s = 1); otherwise it reads row r of src.
+// division.  One warp per row with the row held in registers (VPL 16-byte
+// vectors of 8 bf16 per lane); rows longer than 16*32*8 take two passes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
@@ -134,75 +150,108 @@ __device__ __forceinline__ uint32_t e4m3_pack4(float a, float b, float c, float 
   return qa | (qb << 8) | (qc << 16) | (qd << 24);
 }
 
-__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ src,
-                                                         const int32_t* __restrict__ sorted,
-                                                         const int32_t* __restrict__ num_post, int N, int k,
-                                                         int C, uint2* __restrict__ q, float* __restrict__ scale) {
-  __shared__ float s_red[8];
-  const int np = *num_post;
-  const int vec = C / 8;  // 8 bf16 per uint4 in, 8 codes per uint2 out
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r = blockIdx.x; r < np; r += gridDim.x) {
-    const uint4* row;
-    if (sorted) {
-      const int slot = __ldg(sorted + r);
-      row = slot < N ? src + (long long)(slot / k) * vec : nullptr;
-    } else {
-      row = src + (long long)r * vec;
-    }
-    uint2* dst = q + (long long)r * vec;
-    if (!row) {
-      for (int c = threadIdx.x; c < vec; c += blockDim.x) dst[c] = make_uint2(0, 0);
-      if (threadIdx.x == 0) scale[r] = 1.f;
-      continue;
-    }
+__device__ __forceinline__ float absmax8(const uint4& v) {
+  return fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
+               fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+}
+
+__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
+  uint2 o;
+  o.x = e4m3_pack4(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s), __fdiv_rn(bf16_lo(v.y), s),
+                   __fdiv_rn(bf16_hi(v.y), s));
+  o.y = e4m3_pack4(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s), __fdiv_rn(bf16_lo(v.w), s),
+                   __fdiv_rn(bf16_hi(v.w), s));
+  return o;
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __restrict__ src,
+                                                              const int32_t* __restrict__ nrows_dev, int nrows,
+                                                              int vec, uint2* __restrict__ q,
+                                                              float* __restrict__ scale) {
+  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
+    const uint4* row = src + (long long)r * vec;
+    uint4 v[VPL];
     float amax = 0.f;
-    for (int c = threadIdx.x; c < vec; c += blockDim.x) {
-      const uint4 v = __ldg(row + c);
-      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
-                               fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
-                               fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int c = lane + 32 * i;
+      v[i] = c < vec ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
+      amax = fmaxf(amax, absmax8(v[i]));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) s_red[warp] = amax;
-    __syncthreads();
-    amax = s_red[0];
-    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) amax = fmaxf(amax, s_red[i]);
-    __syncthreads();
     const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    for (int c = threadIdx.x; c < vec; c += blockDim.x) {
-      const uint4 v = __ldg(row + c);
-      uint2 o;
-      o.x = e4m3_pack4(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s), __fdiv_rn(bf16_lo(v.y), s),
-                       __fdiv_rn(bf16_hi(v.y), s));
-      o.y = e4m3_pack4(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s), __fdiv_rn(bf16_lo(v.w), s),
-                       __fdiv_rn(bf16_hi(v.w), s));
-      dst[c] = o;
+    uint2* dst = q + (long long)r * vec;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int c = lane + 32 * i;
+      if (c < vec) dst[c] = quant8(v[i], s);
     }
-    if (threadIdx.x == 0) scale[r] = s;
+    if (lane == 0) scale[r] = s;
   }
 }
 
-static int rows_grid(int P) {
+// Rows longer than the register-resident limit: one warp per row, two passes
+// (the second pass re-reads the row from L1/L2).
+__global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __restrict__ src,
+                                                               const int32_t* __restrict__ nrows_dev, int nrows,
+                                                               int vec, uint2* __restrict__ q,
+                                                               float* __restrict__ scale) {
+  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
+    const uint4* row = src + (long long)r * vec;
+    float amax = 0.f;
+    for (int c = lane; c < vec; c += 32) amax = fmaxf(amax, absmax8(__ldg(row + c)));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint2* dst = q + (long long)r * vec;
+    for (int c = lane; c < vec; c += 32) dst[c] = quant8(__ldg(row + c), s);
+    if (lane == 0) scale[r] = s;
+  }
+}
+
+static int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long long g = (long long)sms * 8;
-  return (int)(P < g ? (P > 0 ? P : 1) : g);
+  return sms;
 }
 
-cudaError_t launch_permute_bf16(const void* x, const int32_t* sorted, const int32_t* num_post, int P, int N,
-                                int k, int H, void* A, cudaStream_t s) {
-  permute_bf16_kernel<<<rows_grid(P), 256, 0, s>>>((const uint4*)x, sorted, num_post, N, k, H, (uint4*)A);
+// grid for one warp per row, 8 warps per CTA, at most 16 CTAs per SM
+static int warp_rows_grid(long long rows) {
+  const long long need = (rows + 7) / 8;
+  const long long cap = (long long)sm_count() * 16;
+  return (int)(need < 1 ? 1 : (need < cap ? need : cap));
+}
+
+cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,
+                               const int32_t* num_post, int P, int N, int k, int row_bytes, void* dst,
+                               float* dst_scale, cudaStream_t s) {
+  gather_rows_kernel<<<warp_rows_grid(P), 256, 0, s>>>((const uint4*)src, src_scale, sorted, num_post, N, k,
+                                                        row_bytes / 16, (uint4*)dst, dst_scale);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, const int32_t* num_post, int P, int N,
-                              int k, int C, void* q, float* scale, cudaStream_t s) {
-  quant_rows_kernel<<<rows_grid(P), 256, 0, s>>>((const uint4*)src, sorted, num_post, N, k, C, (uint2*)q,
-                                                 scale);
+cudaError_t launch_quant_rows(const void* src, const int32_t* nrows_dev, int nrows, int C, void* q, float* scale,
+                              cudaStream_t s) {
+  const int vec = C / 8;
+  const int vpl = (vec + 31) / 32;
+  const int g = warp_rows_grid(nrows);
+  const uint4* in = (const uint4*)src;
+  uint2* out = (uint2*)q;
+  if (vpl <= 1) quant_rows_warp_kernel<1><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+  else if (vpl <= 2) quant_rows_warp_kernel<2><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+  else if (vpl <= 4) quant_rows_warp_kernel<4><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+  else if (vpl <= 8) quant_rows_warp_kernel<8><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+  else if (vpl <= 16) quant_rows_warp_kernel<16><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
   return cudaGetLastError();
 }
 

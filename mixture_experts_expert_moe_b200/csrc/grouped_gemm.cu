@@ -21,8 +21,9 @@
 //     expert -> weight tile -> token group, so CTAs that run at the same
 //     time share weight tiles through L2 when an expert has several groups.
 //   * warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread)
-//     and owns the TMEM allocation, warps 2..5 drain TMEM (tcgen05.ld) and
-//     run the epilogue.  An S-stage shared-memory ring (full/empty
+//     and owns the TMEM allocation, warps 2..9 drain TMEM (tcgen05.ld, two
+//     warps per lane quarter on alternate column chunks) and run the
+//     epilogue.  An S-stage shared-memory ring (full/empty
 //     mbarriers) decouples TMA from MMA; two TMEM accumulator buffers
 //     decouple MMA from the epilogue when they fit in 512 columns.
 //   * every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
@@ -31,7 +32,7 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -331,8 +332,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5 ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------- epilogue: warps 2..9 ----------------
+    // two warps per TMEM lane quarter (a warp may only read lanes 32*(warp%4)..+31);
+    // they take alternate 16-column chunks
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int m = 32 * q + lane;
     int it = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           su = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n);
         }
         __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
-        for (int c = 0; c < ti.nrows; c += 16) {
+        for (int c = 16 * half; c < ti.nrows; c += 32) {
           float g[16], u[16];
           tmem_ld16(tb + c, g);
           tmem_ld16(tb + p.tn + c, u);
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 gv = gv * sa * sg;
                 uv = uv * sa * su;
               }
-              const float hv = gv / (1.f + expf(-gv)) * uv;
+              const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
               h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
             }
           }
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (has1) sw1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
         }
         float* o = reinterpret_cast<float*>(p.out);
-        for (int c = 0; c < ti.nrows; c += 16) {
+        for (int c = 16 * half; c < ti.nrows; c += 32) {
           float v0[16], v1[16];
           tmem_ld16(tb + c, v0);
           if (has1) tmem_ld16(tb + p.tn + c, v1);

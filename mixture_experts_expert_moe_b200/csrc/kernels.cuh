@@ -27,10 +27,15 @@ cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout
 
 cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* ids,
                              float* w, cudaStream_t s);
-cudaError_t launch_permute_bf16(const void* x, const int32_t* sorted, const int32_t* num_post, int P, int N,
-                                int k, int H, void* A, cudaStream_t s);
-cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, const int32_t* num_post, int P, int N,
-                              int k, int C, void* q, float* scale, cudaStream_t s);
+// dst row r = src row sorted[r]/k (row_bytes each, a multiple of 16), zero for
+// padding; with scales also dst_scale[r] = src_scale[token] (1 for padding)
+cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,
+                               const int32_t* num_post, int P, int N, int k, int row_bytes, void* dst,
+                               float* dst_scale, cudaStream_t s);
+// per-row E4M3 quantisation of a bf16 [rows, C] matrix; rows = *nrows_dev if
+// non-null, else nrows
+cudaError_t launch_quant_rows(const void* src, const int32_t* nrows_dev, int nrows, int C, void* q, float* scale,
+                              cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
 
