@@ -4,9 +4,8 @@
 // section "Writing AMD-friendly CUDA code with 3x~7x speed-up"):
 //   (D) distributed concurrent counting: every CTA counts the expert ids of
 //       its contiguous chunk of flat slots.  Inside a CTA every warp owns a
-//       contiguous sub-chunk and a private histogram row in shared memory;
-//       lanes that hold the same expert are grouped with __match_any_sync so
-//       one leader updates the row (no atomics, and the order is fixed).
+//       contiguous sub-chunk and a private histogram row in shared memory
+//       (shared-memory atomics; counting needs no order).
 //   (C) cumulative sums: the warp rows are scanned into per-warp exclusive
 //       prefixes (the article's "unaligned local cumsum"), the CTA totals go
 //       to a global matrix hist[expert][cta] (the "merge" through a
@@ -21,7 +20,11 @@
 //       block) are written by the CTA that owns the block.
 // Unlike the article's design there is no second kernel and no single-block
 // alignment step: every CTA redoes the small E-wide scan itself, which costs
-// less than another launch or grid-wide wait.
+// less than another launch or grid-wide wait.  The same kernel, instantiated
+// with gating in front and the GEMM tile plan behind, is the single routing
+// launch of moe_forward; with one CTA (small batches) it needs no grid-wide
+// wait at all.
+#include "gate.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -95,7 +98,8 @@ __device__ int block_exclusive_scan(int* a, int n) {
 }
 
 // Loads kSub sub-steps (32 consecutive slots each) of a warp's sub-chunk;
-// ids outside [0, E) and slots past the end become -1.
+// ids outside [0, E) and slots past the end become -1.  Plain (L2) loads: in
+// the fused routing kernel the ids were written earlier in the same launch.
 __device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, long long end, int lane, int E,
                                           int (&key)[kSub]) {
   bool bad = false;
@@ -104,7 +108,7 @@ __device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, lo
     const long long i = base + q * 32 + lane;
     int v = -1;
     if (i < end) {
-      v = __ldg(ids + i);
+      v = __ldcg(ids + i);
       if (v < 0 || v >= E) {
         bad = true;
         v = -1;
@@ -115,7 +119,12 @@ __device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, lo
   return bad;
 }
 
-__global__ void __launch_bounds__(kAlignThreads, 1) align_sort_kernel(AlignParams p) {
+// kGate: the CTA first gates the tokens whose slots it owns (its chunk is a
+// multiple of k) and writes ids/weights.  kPlan: CTA 0 finally writes the
+// grouped GEMMs' tile plan from the padded offsets.  With one CTA there is no
+// grid-wide wait.
+template <int EPL, bool kGate, bool kPlan>
+__global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, RouteExtra r) {
   extern __shared__ int smem[];
   const int E = p.E;
   const int G = gridDim.x;
@@ -128,15 +137,23 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_sort_kernel(AlignParam
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kAlignWarps * E; i += blockDim.x) wcnt[i] = 0;
   if (tid == 0) s_bad = 0;
-  __syncthreads();
 
   const long long cta_begin = (long long)blockIdx.x * p.chunk;
+  if (kGate) {
+    // ---- gating of this CTA's tokens (warp per token) ----------------------
+    const long long t0 = cta_begin / r.k;
+    const long long t1 = min((long long)r.T, (cta_begin + p.chunk) / r.k);
+    for (long long t = t0 + warp; t < t1; t += kAlignWarps)
+      gate_token<EPL>(r.logits, r.bias, t, E, r.k, r.ids_out, r.w_out, lane);
+  }
+  __syncthreads();
+
   const int wsub = p.chunk / kAlignWarps;
   const long long w_begin = cta_begin + (long long)warp * wsub;
   const long long w_end = min((long long)p.N, w_begin + wsub);
   int* my = wcnt + warp * E;
 
-  // ---- (D) count: each warp into its own row -------------------------------
+  // ---- (D) count: each warp into its own row (shared-memory atomics) -----
   bool bad = false;
   for (long long base = w_begin; base < w_end; base += 32 * kSub) {
     int key[kSub];
@@ -158,46 +175,52 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_sort_kernel(AlignParam
       wcnt[w * E + e] = run;
       run += c;
     }
-    p.hist[(long long)e * G + blockIdx.x] = run;
-  }
-
-  if (!grid_wait(p.barrier, p.expected, p.timeout_ns)) {
-    if (tid == 0) dev_flag(p.status, MOE_DEV_TIMEOUT);
-    return;
-  }
-
-  // ---- (C) own prefix and expert totals from row e of hist ------------------
-  // warp w reduces experts w, w+32, ...; lane l reads CTAs l, l+32, ...
-  for (int e0 = warp; e0 < E; e0 += kAlignWarps * 8) {
-    int pre[8], tot[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) pre[u] = tot[u] = 0;
-    for (int c = 0; c < G; c += 32) {
-      const int b = c + lane;
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * kAlignWarps;
-        v[u] = (e < E && b < G) ? __ldcg(p.hist + (long long)e * G + b) : 0;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        pre[u] += b < (int)blockIdx.x ? v[u] : 0;
-        tot[u] += v[u];
-      }
+    if (G > 1) p.hist[(long long)e * G + blockIdx.x] = run;
+    else {
+      s_tot[e] = run;
+      s_base[e] = 0;
+      s_off[e] = (run + p.bm - 1) / p.bm * p.bm;
     }
+  }
+
+  if (G > 1) {
+    if (!grid_wait(p.barrier, p.expected, p.timeout_ns)) {
+      if (tid == 0) dev_flag(p.status, MOE_DEV_TIMEOUT);
+      return;
+    }
+    // ---- (C) own prefix and expert totals from row e of hist ----------------
+    // warp w reduces experts w, w+32, ...; lane l reads CTAs l, l+32, ...
+    for (int e0 = warp; e0 < E; e0 += kAlignWarps * 8) {
+      int pre[8], tot[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 8; ++u) pre[u] = tot[u] = 0;
+      for (int c = 0; c < G; c += 32) {
+        const int b = c + lane;
+        int v[8];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        pre[u] += __shfl_xor_sync(0xffffffffu, pre[u], off);
-        tot[u] += __shfl_xor_sync(0xffffffffu, tot[u], off);
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + u * kAlignWarps;
+          v[u] = (e < E && b < G) ? __ldcg(p.hist + (long long)e * G + b) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          pre[u] += b < (int)blockIdx.x ? v[u] : 0;
+          tot[u] += v[u];
+        }
       }
-      const int e = e0 + u * kAlignWarps;
-      if (lane == 0 && e < E) {
-        s_tot[e] = tot[u];
-        s_base[e] = pre[u];
-        s_off[e] = (tot[u] + p.bm - 1) / p.bm * p.bm;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          pre[u] += __shfl_xor_sync(0xffffffffu, pre[u], off);
+          tot[u] += __shfl_xor_sync(0xffffffffu, tot[u], off);
+        }
+        const int e = e0 + u * kAlignWarps;
+        if (lane == 0 && e < E) {
+          s_tot[e] = tot[u];
+          s_base[e] = pre[u];
+          s_off[e] = (tot[u] + p.bm - 1) / p.bm * p.bm;
+        }
       }
     }
   }
@@ -242,11 +265,47 @@ __global__ void __launch_bounds__(kAlignThreads, 1) align_sort_kernel(AlignParam
       __syncwarp();
     }
   }
+
+  if (kPlan && blockIdx.x == 0) {
+    // ---- tile plan of the grouped GEMMs (layout in kernels.cuh) --------------
+    __syncthreads();
+    int* s_pg = wcnt;              // tiles per expert -> exclusive prefix
+    int* s_pd = wcnt + E + 1;
+    for (int e = tid; e < E; e += blockDim.x) {
+      const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+      const int g = (rows + r.tn - 1) / r.tn;
+      r.plan[4 + e] = s_off[e];
+      r.plan[4 + E + e] = rows;
+      r.plan[4 + 2 * E + e] = g;
+      s_pg[e] = g * r.nw_gu;
+      s_pd[e] = g * r.nw_dn;
+    }
+    __syncthreads();
+    const int tg = block_exclusive_scan(s_pg, E);
+    const int td = block_exclusive_scan(s_pd, E);
+    for (int e = tid; e < E; e += blockDim.x) {
+      r.plan[4 + 3 * E + e] = s_pg[e];
+      r.plan[5 + 4 * E + e] = s_pd[e];
+    }
+    if (tid == 0) {
+      r.plan[4 + 4 * E] = tg;
+      r.plan[5 + 5 * E] = td;
+      r.plan[0] = tg;
+      r.plan[1] = td;
+      r.plan[2] = r.tn;
+      r.plan[3] = total_post;
+    }
+  }
 }
 
 size_t align_smem_bytes(int E) { return (size_t)(kAlignWarps + 3) * E * sizeof(int); }
 
-cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream) {
+template <typename K>
+static cudaError_t launch_route_impl(K kernel, const AlignParams& p, const RouteExtra& r, int grid,
+                                     cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)align_smem_bytes(1024));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kAlignThreads);
@@ -257,7 +316,22 @@ cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t strea
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, align_sort_kernel, p);
+  return cudaLaunchKernelEx(&cfg, kernel, p, r);
+}
+
+cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream) {
+  RouteExtra r = {};
+  return launch_route_impl(route_kernel<1, false, false>, p, r, grid, stream);
+}
+
+cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream) {
+  const int epl = (p.E + 31) / 32;
+  if (epl <= 1) return launch_route_impl(route_kernel<1, true, true>, p, r, grid, stream);
+  if (epl <= 2) return launch_route_impl(route_kernel<2, true, true>, p, r, grid, stream);
+  if (epl <= 4) return launch_route_impl(route_kernel<4, true, true>, p, r, grid, stream);
+  if (epl <= 8) return launch_route_impl(route_kernel<8, true, true>, p, r, grid, stream);
+  if (epl <= 16) return launch_route_impl(route_kernel<16, true, true>, p, r, grid, stream);
+  return launch_route_impl(route_kernel<32, true, true>, p, r, grid, stream);
 }
 
 // Largest cooperative grid: one CTA per SM (the column reads of phase C grow
@@ -275,9 +349,9 @@ int align_max_ctas(int E, int* err_out) {
   int sms = 0, per_sm = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(align_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+    e = cudaFuncSetAttribute(route_kernel<32, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, align_sort_kernel, kAlignThreads, need);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_kernel<32, true, true>, kAlignThreads, need);
   *err_out = (int)e;
   if (e != cudaSuccess || per_sm < 1) return 0;
   (void)E;

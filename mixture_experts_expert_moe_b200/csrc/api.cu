@@ -55,6 +55,9 @@ moe_status_t check_device() {
 // ---------------------------------------------------------------------------
 constexpr int kMaxAlignCtas = 1024;
 constexpr int kMinSlotsPerCta = 4096;
+// up to this many slots the FP8 path quantises per sorted row (the token's k
+// copies are quantised redundantly) instead of once per token plus a gather
+constexpr int kFusedQuantSlots = 4096;
 
 bool align_args_ok(int T, int k, int E, int bm) {
   return T >= 0 && k >= 1 && E >= 1 && E <= 1024 && bm >= 1 && bm <= 1024 &&
@@ -165,7 +168,8 @@ moe_status_t gemm_fail(int r, const char* what) {
 // Runs plan -> gather(+quant) -> gate/up GEMM -> (requant) -> down GEMM.
 moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
                      const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
-                     float* y, uint8_t* ws, int32_t* status, cudaStream_t stream, void** ev = nullptr) {
+                     float* y, uint8_t* ws, int32_t* status, cudaStream_t stream, void** ev = nullptr,
+                     bool plan_ready = false) {
   const FfnWs L = ffn_ws_layout(s);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
@@ -177,11 +181,16 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   float* sH = reinterpret_cast<float*>(ws + L.sH);
   const int P = (int)s.P, N = (int)s.N;
 
-  MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status, stream));
+  if (!plan_ready)
+    MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status,
+                            stream));
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
-  if (s.fp8) {
+  if (s.fp8 && N <= kFusedQuantSlots) {
+    // few slots: each sorted row quantises its token directly (one launch)
+    MOE_CU(moe::launch_quant_rows(x, sorted, N, s.k, num_post, P, s.H, A, sA, stream));
+  } else if (s.fp8) {
     // quantise each token once, then gather codes and scales into sorted order
-    MOE_CU(moe::launch_quant_rows(x, nullptr, s.T, s.H, xq, sx, stream));
+    MOE_CU(moe::launch_quant_rows(x, nullptr, N, s.k, nullptr, s.T, s.H, xq, sx, stream));
     MOE_CU(moe::launch_gather_rows(xq, sx, sorted, num_post, P, N, s.k, s.H, A, sA, stream));
   } else {
     MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, P, N, s.k, s.H * 2, A, nullptr, stream));
@@ -212,7 +221,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
 
-  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, num_post, P, s.I, hq, sH, stream));
+  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, nullptr, N, s.k, num_post, P, s.I, hq, sH, stream));
   MOE_CU(record(ev, MOE_STAGE_REQUANT + 1, stream));
 
   moe::GemmLaunch g2 = {};
@@ -238,6 +247,62 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
+  return MOE_OK;
+}
+
+// Gate + align&sort + tile plan in one launch (moe_forward).
+moe_status_t run_route(const FfnShape& s, const float* logits, const float* bias, int32_t* ids, float* w,
+                       int32_t* sorted, int32_t* expert_ids, int32_t* num_post, void* align_ws, int32_t* plan,
+                       int32_t* status, cudaStream_t stream) {
+  const int N = (int)s.N;
+  int err = 0;
+  const int max_ctas = moe::align_max_ctas(s.E, &err);
+  if (err) return cuda_fail((cudaError_t)err, "route occupancy");
+  if (max_ctas < 1) return MOE_ERR_UNSUPPORTED;
+  int g = 1024, b = s.k;  // unit = lcm(32 warps x 32 lanes, k): a CTA's slots are whole tokens
+  while (b) {
+    const int t = g % b;
+    g = b;
+    b = t;
+  }
+  const int unit = 1024 / g * s.k;
+  int grid = (int)(((long long)N + kMinSlotsPerCta - 1) / kMinSlotsPerCta);
+  grid = grid < 1 ? 1 : grid;
+  grid = grid > max_ctas ? max_ctas : grid;
+  grid = grid > kMaxAlignCtas ? kMaxAlignCtas : grid;
+  long long chunk = ((long long)N + grid - 1) / grid;
+  chunk = (chunk + unit - 1) / unit * unit;
+  if (chunk < unit) chunk = unit;
+  grid = N > 0 ? (int)((N + chunk - 1) / chunk) : 1;
+
+  uint8_t* wsb = static_cast<uint8_t*>(align_ws);
+  moe::AlignParams p;
+  p.ids = ids;
+  p.N = N;
+  p.E = s.E;
+  p.bm = s.bm;
+  p.chunk = (int)chunk;
+  p.sorted = sorted;
+  p.expert_ids = expert_ids;
+  p.num_post = num_post;
+  p.barrier = reinterpret_cast<int*>(wsb);
+  p.hist = reinterpret_cast<int32_t*>(wsb + 256);
+  p.status = status;
+  p.timeout_ns = moe::kDefaultTimeoutNs;
+  p.expected = grid;
+  moe::RouteExtra r;
+  r.logits = logits;
+  r.bias = bias;
+  r.T = s.T;
+  r.k = s.k;
+  r.ids_out = ids;
+  r.w_out = w;
+  r.plan = plan;
+  r.tn = s.tn;
+  r.nw_gu = s.I / 128;
+  r.nw_dn = (s.H + 255) / 256;
+  if (grid > 1) MOE_CU(cudaMemsetAsync(p.barrier, 0, sizeof(int), stream));
+  MOE_CU(moe::launch_route(p, r, grid, stream));
   return MOE_OK;
 }
 
@@ -390,13 +455,15 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   void** ev = a->stage_events;
   float* y = reinterpret_cast<float*>(w + L.y);
   MOE_CU(record(ev, 0, cs));
-  MOE_CU(moe::launch_topk_gate(a->logits, a->bias, s.T, s.E, s.k, ids, tw, cs));
-  MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
-  st = run_align(ids, s.T, s.k, s.E, s.bm, sorted, eids, npost, w + L.align, dev_status, cs);
+  // gate, align&sort and the GEMM tile plan are one launch: stages 0..2 end together
+  uint8_t* ffn_ws = w + L.ffn;
+  int32_t* plan = reinterpret_cast<int32_t*>(ffn_ws + ffn_ws_layout(s).plan);
+  st = run_route(s, a->logits, a->bias, ids, tw, sorted, eids, npost, w + L.align, plan, dev_status, cs);
   if (st) return st;
+  MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
-  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, y, w + L.ffn, dev_status,
-               cs, ev);
+  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, y, ffn_ws, dev_status,
+               cs, ev, /*plan_ready=*/true);
   if (st) return st;
   MOE_CU(moe::launch_combine(y, tw, s.T, s.k, s.H, a->out, a->out_dtype == MOE_BF16, cs));
   MOE_CU(record(ev, MOE_STAGE_COMBINE + 1, cs));

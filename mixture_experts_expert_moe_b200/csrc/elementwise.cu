@@ -7,74 +7,22 @@
 //   combine        top-k weighted sum of the per-slot expert outputs
 #include <cfloat>
 
+#include "gate.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Top-k gating (MoE Align & Sort article, "FasterTransformer":
-// moe_softmax + moe_top_k fused as topk_gating_softmax).  Lane l holds the
-// logits of experts l, l+32, ...; k rounds of a warp arg-max (ties to the
-// lower expert index) pick the experts in descending order.  The weights are
-// exp(l_j - l_max) over the chosen experts, normalised by their sum, which is
-// softmax over all E renormalised over the chosen k.
+// Top-k gating, one warp per token (the per-token work is gate_token in
+// gate.cuh).
 // ---------------------------------------------------------------------------
 template <int EPL>
 __global__ void __launch_bounds__(256) topk_gate_kernel(const float* __restrict__ logits,
                                                         const float* __restrict__ bias, int T, int E, int k,
                                                         int32_t* __restrict__ ids, float* __restrict__ w) {
-  const int lane = threadIdx.x & 31;
   const long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  float v[EPL];
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = -FLT_MAX;
-    if (e < E) {
-      float x = __ldg(logits + t * E + e);
-      if (bias) x = __fadd_rn(x, __ldg(bias + e));
-      v[j] = x;
-    }
-  }
-  uint32_t taken = 0;
-  float my_val = 0.f;
-  int my_id = 0;
-  for (int r = 0; r < k; ++r) {
-    float best = -FLT_MAX;
-    int be = INT_MAX;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && (be == INT_MAX || v[j] > best)) {
-        best = v[j];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (oe != INT_MAX && (be == INT_MAX || ob > best || (ob == best && oe < be))) {
-        best = ob;
-        be = oe;
-      }
-    }
-    if (lane == (be & 31)) taken |= 1u << (be >> 5);
-    if (lane == r) {
-      my_val = best;
-      my_id = be;
-    }
-  }
-  const float top = __shfl_sync(0xffffffffu, my_val, 0);
-  const float ex = lane < k ? expf(my_val - top) : 0.f;
-  float sum = ex;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-  if (lane < k) {
-    ids[t * k + lane] = my_id;
-    w[t * k + lane] = __fdiv_rn(ex, sum);
-  }
+  gate_token<EPL>(logits, bias, t, E, k, ids, w, threadIdx.x & 31);
 }
 
 cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* ids,
@@ -137,7 +85,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 // GC-MoE: requantisation between the GEMMs).  s = amax / 448 in fp32 (1 for
 // an all-zero row); code = e4m3_rne_satfinite(v / s) with an IEEE fp32
 // division.  One warp per row with the row held in registers (VPL 16-byte
-// vectors of 8 bf16 per lane); rows longer than 16*32*8 take two passes.
+// vectors of 8 bf16 per lane); rows longer than 16*32*8 take two passes.  With
+// a row map the kernel also gathers (sorted row r quantises its token).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
@@ -164,8 +113,17 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
   return o;
 }
 
+// gather (optional): row r quantises token sorted[r] / k of src (padding
+// rows: zero codes, scale 1) instead of src row r.
+__device__ __forceinline__ long long quant_src_row(const int32_t* sorted, int r, int N, int k) {
+  if (!sorted) return r;
+  const int slot = __ldg(sorted + r);
+  return slot < N ? slot / k : -1;
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __restrict__ src,
+                                                              const int32_t* __restrict__ sorted, int N, int k,
                                                               const int32_t* __restrict__ nrows_dev, int nrows,
                                                               int vec, uint2* __restrict__ q,
                                                               float* __restrict__ scale) {
@@ -173,7 +131,14 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
-    const uint4* row = src + (long long)r * vec;
+    const long long sr = quant_src_row(sorted, r, N, k);
+    uint2* dst = q + (long long)r * vec;
+    if (sr < 0) {
+      for (int c = lane; c < vec; c += 32) dst[c] = make_uint2(0, 0);
+      if (lane == 0) scale[r] = 1.f;
+      continue;
+    }
+    const uint4* row = src + sr * vec;
     uint4 v[VPL];
     float amax = 0.f;
 #pragma unroll
@@ -185,7 +150,6 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    uint2* dst = q + (long long)r * vec;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int c = lane + 32 * i;
@@ -198,6 +162,7 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
 // Rows longer than the register-resident limit: one warp per row, two passes
 // (the second pass re-reads the row from L1/L2).
 __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __restrict__ src,
+                                                               const int32_t* __restrict__ sorted, int N, int k,
                                                                const int32_t* __restrict__ nrows_dev, int nrows,
                                                                int vec, uint2* __restrict__ q,
                                                                float* __restrict__ scale) {
@@ -205,13 +170,19 @@ __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __re
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
-    const uint4* row = src + (long long)r * vec;
+    const long long sr = quant_src_row(sorted, r, N, k);
+    uint2* dst = q + (long long)r * vec;
+    if (sr < 0) {
+      for (int c = lane; c < vec; c += 32) dst[c] = make_uint2(0, 0);
+      if (lane == 0) scale[r] = 1.f;
+      continue;
+    }
+    const uint4* row = src + sr * vec;
     float amax = 0.f;
     for (int c = lane; c < vec; c += 32) amax = fmaxf(amax, absmax8(__ldg(row + c)));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    uint2* dst = q + (long long)r * vec;
     for (int c = lane; c < vec; c += 32) dst[c] = quant8(__ldg(row + c), s);
     if (lane == 0) scale[r] = s;
   }
@@ -239,19 +210,21 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_rows(const void* src, const int32_t* nrows_dev, int nrows, int C, void* q, float* scale,
-                              cudaStream_t s) {
+cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
+                              int nrows, int C, void* q, float* scale, cudaStream_t s) {
   const int vec = C / 8;
   const int vpl = (vec + 31) / 32;
   const int g = warp_rows_grid(nrows);
   const uint4* in = (const uint4*)src;
   uint2* out = (uint2*)q;
-  if (vpl <= 1) quant_rows_warp_kernel<1><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
-  else if (vpl <= 2) quant_rows_warp_kernel<2><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
-  else if (vpl <= 4) quant_rows_warp_kernel<4><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
-  else if (vpl <= 8) quant_rows_warp_kernel<8><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
-  else if (vpl <= 16) quant_rows_warp_kernel<16><<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
-  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, nrows_dev, nrows, vec, out, scale);
+#define MOE_QUANT(V) quant_rows_warp_kernel<V><<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale)
+  if (vpl <= 1) MOE_QUANT(1);
+  else if (vpl <= 2) MOE_QUANT(2);
+  else if (vpl <= 4) MOE_QUANT(4);
+  else if (vpl <= 8) MOE_QUANT(8);
+  else if (vpl <= 16) MOE_QUANT(16);
+  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
+#undef MOE_QUANT
   return cudaGetLastError();
 }
 

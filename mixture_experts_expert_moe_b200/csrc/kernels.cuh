@@ -20,8 +20,21 @@ struct AlignParams {
   int expected;     // arrivals to wait for (gridDim.x; larger only in the timeout test)
 };
 
+// Extra inputs of the fused routing launch (gating in front, tile plan behind).
+struct RouteExtra {
+  const float* logits;  // [T, E]
+  const float* bias;    // [E] or null
+  int T, k;
+  int32_t* ids_out;     // [T*k] (the same buffer AlignParams::ids reads)
+  float* w_out;         // [T*k]
+  int32_t* plan;        // plan layout below
+  int tn, nw_gu, nw_dn;
+};
+
 size_t align_smem_bytes(int E);
 cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream);
+// gate + align&sort + tile plan in one cooperative launch (p.chunk % k == 0)
+cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream);
 int align_max_ctas(int E, int* err_out);
 cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout_ns, cudaStream_t stream);
 
@@ -32,10 +45,11 @@ cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int 
 cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,
                                const int32_t* num_post, int P, int N, int k, int row_bytes, void* dst,
                                float* dst_scale, cudaStream_t s);
-// per-row E4M3 quantisation of a bf16 [rows, C] matrix; rows = *nrows_dev if
-// non-null, else nrows
-cudaError_t launch_quant_rows(const void* src, const int32_t* nrows_dev, int nrows, int C, void* q, float* scale,
-                              cudaStream_t s);
+// per-row E4M3 quantisation of bf16 rows of length C; rows = *nrows_dev if
+// non-null, else nrows.  With `sorted`, output row r quantises source row
+// sorted[r] / k (zero codes, scale 1 for padding slots >= N).
+cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
+                              int nrows, int C, void* q, float* scale, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
 
