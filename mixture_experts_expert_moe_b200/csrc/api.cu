@@ -58,6 +58,8 @@ constexpr int kMinSlotsPerCta = 4096;
 // up to this many slots the FP8 path quantises per sorted row (the token's k
 // copies are quantised redundantly) instead of once per token plus a gather
 constexpr int kFusedQuantSlots = 4096;
+// tokens gated per CTA of the fused routing launch
+constexpr int kRouteTokensPerCta = 64;
 
 bool align_args_ok(int T, int k, int E, int bm) {
   return T >= 0 && k >= 1 && E >= 1 && E <= 1024 && bm >= 1 && bm <= 1024 &&
@@ -259,14 +261,15 @@ moe_status_t run_route(const FfnShape& s, const float* logits, const float* bias
   const int max_ctas = moe::align_max_ctas(s.E, &err);
   if (err) return cuda_fail((cudaError_t)err, "route occupancy");
   if (max_ctas < 1) return MOE_ERR_UNSUPPORTED;
-  int g = 1024, b = s.k;  // unit = lcm(32 warps x 32 lanes, k): a CTA's slots are whole tokens
+  int g = 32, b = s.k;  // unit = lcm(32 warps, k): a CTA's slots are whole tokens
   while (b) {
     const int t = g % b;
     g = b;
     b = t;
   }
-  const int unit = 1024 / g * s.k;
-  int grid = (int)(((long long)N + kMinSlotsPerCta - 1) / kMinSlotsPerCta);
+  const int unit = 32 / g * s.k;
+  // the gating work is per token: spread the tokens over the SMs
+  int grid = (s.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
   grid = grid < 1 ? 1 : grid;
   grid = grid > max_ctas ? max_ctas : grid;
   grid = grid > kMaxAlignCtas ? kMaxAlignCtas : grid;
