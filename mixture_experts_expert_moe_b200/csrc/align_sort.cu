@@ -98,23 +98,25 @@ __device__ int block_exclusive_scan(int* a, int n) {
 }
 
 // Loads kSub sub-steps (32 consecutive slots each) of a warp's sub-chunk;
-// ids outside [0, E) and slots past the end become -1.  Plain (L2) loads: in
-// the fused routing kernel the ids were written earlier in the same launch.
+// ids outside [0, E) and slots past the end become -1.  All loads are issued
+// before any value is used (a use right after a load would expose every load
+// latency in turn).  Plain (L2) loads: in the fused routing kernel the ids
+// were written earlier in the same launch.
 __device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, long long end, int lane, int E,
                                           int (&key)[kSub]) {
+#pragma unroll
+  for (int q = 0; q < kSub; ++q) {
+    const long long i = base + q * 32 + lane;
+    key[q] = i < end ? __ldcg(ids + i) : -1;
+  }
   bool bad = false;
 #pragma unroll
   for (int q = 0; q < kSub; ++q) {
     const long long i = base + q * 32 + lane;
-    int v = -1;
-    if (i < end) {
-      v = __ldcg(ids + i);
-      if (v < 0 || v >= E) {
-        bad = true;
-        v = -1;
-      }
+    if (i < end && (key[q] < 0 || key[q] >= E)) {
+      bad = true;
+      key[q] = -1;
     }
-    key[q] = v;
   }
   return bad;
 }
@@ -235,21 +237,23 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   const int bpc = (nblk + G - 1) / G;
   const int j0 = blockIdx.x * bpc;
   const int j1 = min(nblk, j0 + bpc);
-  for (int j = j0 + tid; j < j1; j += blockDim.x) {
+  for (int j = j0 + warp; j < j1; j += kAlignWarps) {   // one warp per block
     const int pos = j * p.bm;
     int lo = 0, hi = E - 1;  // last expert whose segment starts at or before pos
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
     }
-    p.expert_ids[j] = lo;
+    if (lane == 0) p.expert_ids[j] = lo;
     const int fill = s_off[lo] + s_tot[lo];  // first padding position of expert lo
-    for (int q = max(fill, pos); q < pos + p.bm; ++q) p.sorted[q] = p.N;
+    for (int q = max(fill, pos) + lane; q < pos + p.bm; q += 32) p.sorted[q] = p.N;
   }
 
   // ---- (P) stable placement ------------------------------------------------
+  // The shared-memory rank chain needs a warp barrier per sub-step; the global
+  // stores are issued after the chain so those barriers do not wait on them.
   for (long long base = w_begin; base < w_end; base += 32 * kSub) {
-    int key[kSub];
+    int key[kSub], dest[kSub];
     load_keys(p.ids, base, w_end, lane, E, key);
 #pragma unroll
     for (int q = 0; q < kSub; ++q) {
@@ -257,13 +261,17 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
       const unsigned peers = __match_any_sync(0xffffffffu, kq);
       const int cnt = kq >= 0 ? my[kq] : 0;
       __syncwarp();
+      dest[q] = -1;
       if (kq >= 0) {
         const unsigned below = peers & lanemask_lt();
-        p.sorted[s_base[kq] + cnt + __popc(below)] = (int)(base + q * 32 + lane);
+        dest[q] = s_base[kq] + cnt + __popc(below);
         if (below == 0) my[kq] = cnt + __popc(peers);
       }
       __syncwarp();
     }
+#pragma unroll
+    for (int q = 0; q < kSub; ++q)
+      if (dest[q] >= 0) p.sorted[dest[q]] = (int)(base + q * 32 + lane);
   }
 
   if (kPlan && blockIdx.x == 0) {

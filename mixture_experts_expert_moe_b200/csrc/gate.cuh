@@ -20,16 +20,18 @@ template <int EPL>
 __device__ __forceinline__ void gate_token(const float* __restrict__ logits, const float* __restrict__ bias,
                                            long long t, int E, int k, int32_t* __restrict__ ids,
                                            float* __restrict__ w, int lane) {
-  float v[EPL];
+  float v[EPL], b[EPL];
+  // all loads first, then the adds (a use right after a load would serialise them)
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = lane + 32 * j;
-    v[j] = -FLT_MAX;
-    if (e < E) {
-      float x = __ldg(logits + t * E + e);
-      if (bias) x = __fadd_rn(x, __ldg(bias + e));
-      v[j] = x;
-    }
+    v[j] = e < E ? __ldg(logits + t * E + e) : -FLT_MAX;
+    b[j] = (bias && e < E) ? __ldg(bias + e) : 0.f;
+  }
+  if (bias) {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (lane + 32 * j < E) v[j] = __fadd_rn(v[j], b[j]);
   }
   uint32_t taken = 0;
   float my_val = 0.f;

@@ -356,16 +356,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
         for (int c = 16 * half; c < ti.nrows; c += 32) {
           float g[16], u[16];
+          // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
+          const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
           tmem_ld16(tb + c, g);
           tmem_ld16(tb + p.tn + c, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int j = c + i;
+            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
             if (j < ti.nrows) {
               const int row = ti.r0 + j;
               float gv = g[i], uv = u[i];
               if (p.fp8) {
-                const float sa = __ldg(p.a_scale + row);
                 gv = gv * sa * sg;
                 uv = uv * sa * su;
               }
@@ -386,16 +388,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float* o = reinterpret_cast<float*>(p.out);
         for (int c = 16 * half; c < ti.nrows; c += 32) {
           float v0[16], v1[16];
+          // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
+          const bool in = lane < 16 && c + lane < ti.nrows;
+          const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
+          const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
           tmem_ld16(tb + c, v0);
           if (has1) tmem_ld16(tb + p.tn + c, v1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int j = c + i;
-            if (j < ti.nrows) {
-              const int row = ti.r0 + j;
-              const int slot = __ldg(p.sorted + row);
+            const int slot = __shfl_sync(0xffffffffu, slot_l, i);
+            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
+            if (c + i < ti.nrows) {
               if (slot < p.n_slots) {
-                const float sa = p.fp8 ? __ldg(p.a_scale + row) : 1.f;
                 float* yr = o + (long long)slot * p.n_out;
                 yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
                 if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
