@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/moe_b200.h: argument checks,
 // workspace carving and kernel launches.  No device memory is allocated and
 // no call synchronises the host.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -111,7 +112,35 @@ moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t*
 struct FfnShape {
   int T, H, I, E, k, bm, fp8, tn;
   long long P, NB, N;
+  int sp_gu, sp_dn;                 // K splits of the two GEMMs
+  long long tiles_gu, tiles_dn;     // upper bounds on the GEMMs' tile counts
 };
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// K splits for a GEMM with about est_tiles tiles of nk k-blocks: when the
+// tiles cannot fill the SMs several times over, split K so the last wave is
+// nearly full (each split keeps at least 4 k-blocks).
+int pick_splits(double est_tiles, int nk, int sms) {
+  if (est_tiles >= 4.0 * sms || est_tiles < 1) return 1;
+  int best = 1;
+  double best_score = -1;
+  const int max_s = nk / 4 < 16 ? nk / 4 : 16;
+  for (int sp = 1; sp <= (max_s > 1 ? max_s : 1); ++sp) {
+    const double units = est_tiles * sp;
+    const double waves = ceil(units / sms);
+    const double score = units / (waves * sms) - 0.01 * (sp - 1);
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = sp;
+    }
+  }
+  return best;
+}
 
 int pick_tn(const FfnShape& s, int hint) {
   if (hint) return hint;
@@ -137,11 +166,25 @@ moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, in
   s->NB = (s->P + bm - 1) / bm;
   s->tn = pick_tn(*s, hint);
   if ((long long)s->P * (s->H > s->I ? s->H : s->I) >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
+  // tile-count bound: every touched expert pads by < bm rows and splits into tn-row groups
+  const long long touched_max = s->N < s->E ? s->N : s->E;
+  const long long groups_max = (s->N + s->tn - 1) / s->tn + touched_max * ((s->bm - 1 + s->tn - 1) / s->tn + 1);
+  s->tiles_gu = groups_max * (s->I / 128);
+  s->tiles_dn = groups_max * ((s->H + 255) / 256);
+  // expected tiles under uniform routing (one group per touched expert when tn covers it)
+  const double touched = s->E * (1.0 - pow(1.0 - 1.0 / s->E, (double)s->N));
+  const double rows = (double)s->N / (touched > 0 ? touched : 1);
+  const double padded = ceil(rows / s->bm) * s->bm;
+  const double groups = touched * ceil(padded / s->tn);
+  const int eb = s->fp8 ? 1 : 2;
+  const int sms = device_sms();
+  s->sp_gu = pick_splits(groups * (s->I / 128), s->H * eb / 128, sms);
+  s->sp_dn = pick_splits(groups * ((s->H + 255) / 256), s->I * eb / 128, sms);
   return MOE_OK;
 }
 
 struct FfnWs {
-  size_t plan, xq, sx, A, sA, h, hq, sH, total;
+  size_t plan, xq, sx, A, sA, h, hq, sH, part_gu, cnt_gu, part_dn, cnt_dn, total;
 };
 
 FfnWs ffn_ws_layout(const FfnShape& s) {
@@ -155,6 +198,11 @@ FfnWs ffn_ws_layout(const FfnShape& s) {
   w.h = c.take((size_t)s.P * s.I * 2);
   w.hq = c.take(s.fp8 ? (size_t)s.P * s.I : 0);
   w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
+  const size_t unit = (size_t)2 * s.tn * 128 * sizeof(float);
+  w.part_gu = c.take(s.sp_gu > 1 ? (size_t)s.tiles_gu * s.sp_gu * unit : 0);
+  w.cnt_gu = c.take(s.sp_gu > 1 ? (size_t)s.tiles_gu * 4 : 0);
+  w.part_dn = c.take(s.sp_dn > 1 ? (size_t)s.tiles_dn * s.sp_dn * unit : 0);
+  w.cnt_dn = c.take(s.sp_dn > 1 ? (size_t)s.tiles_dn * 4 : 0);
   w.total = c.off;
   return w;
 }
@@ -219,6 +267,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g1.p.splits = s.sp_gu;
+  g1.p.part = reinterpret_cast<float*>(ws + L.part_gu);
+  g1.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_gu);
+  if (s.sp_gu > 1) MOE_CU(cudaMemsetAsync(g1.p.tile_cnt, 0, (size_t)s.tiles_gu * 4, stream));
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -246,6 +298,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g2.p.splits = s.sp_dn;
+  g2.p.part = reinterpret_cast<float*>(ws + L.part_dn);
+  g2.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_dn);
+  if (s.sp_dn > 1) MOE_CU(cudaMemsetAsync(g2.p.tile_cnt, 0, (size_t)s.tiles_dn * 4, stream));
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));

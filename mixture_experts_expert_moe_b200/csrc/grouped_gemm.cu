@@ -153,6 +153,60 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
 // the token group has (rounded up to x_box).
 __device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
 
+// Final math of 16 token columns [c, c+16) of a gate/up tile for weight row
+// m of the tile (output feature n): h = bf16(silu(g*scale) * (u*scale)).
+__device__ __forceinline__ void epi_gateup(const GemmParams& p, const TileInfo& ti, int c, int n, float sg, float su,
+                                           const float (&g)[16], const float (&u)[16], int lane) {
+  // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
+  const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
+    if (c + i < ti.nrows) {
+      float gv = g[i], uv = u[i];
+      if (p.fp8) {
+        gv = gv * sa * sg;
+        uv = uv * sa * su;
+      }
+      const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
+      h[(long long)(ti.r0 + c + i) * p.n_out + n] = __float2bfloat16_rn(hv);
+    }
+  }
+}
+
+// Final math of 16 token columns of a down tile: y[slot, n0|n1] = acc * scales.
+__device__ __forceinline__ void epi_down(const GemmParams& p, const TileInfo& ti, int c, int n0, int n1, bool has1,
+                                         float sw0, float sw1, const float (&v0)[16], const float (&v1)[16],
+                                         int lane) {
+  // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
+  const bool in = lane < 16 && c + lane < ti.nrows;
+  const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
+  const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
+  float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int slot = __shfl_sync(0xffffffffu, slot_l, i);
+    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
+    if (c + i < ti.nrows && slot < p.n_slots) {
+      float* yr = o + (long long)slot * p.n_out;
+      yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
+      if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
+    }
+  }
+}
+
+// Barrier of the eight epilogue warps on an mbarrier (8 arrivals), bounded
+// like every other wait; `parity` alternates per use.
+__device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& parity, long long timeout_ns,
+                                         volatile int* abort_flag, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = wait_or_abort(bar, parity, timeout_ns, abort_flag);
+  parity ^= 1u;
+  return ok;
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         GemmParams p) {
@@ -169,8 +223,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = bars + 2 * p.stages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ebar = drain + 1;   // epilogue-warp barrier (split K)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ebar + 1);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
+  int* s_last = s_abort + 1;
   int* s_start = s_abort + 3;   // keep 16-byte alignment of the arrays below
   int* s_rows = s_start + E;
   int* s_groups = s_rows + E;
@@ -188,6 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
+    mbar_init(ebar, 8);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
@@ -214,6 +271,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
   const int cols_per_acc = 2 * p.tn;
   const int xb = x_box_rows(p.tn);
+  // work unit u = (tile u / S, K split u % S); splits of a tile are adjacent
+  const int S = p.splits;
+  const int n_units = n_tiles * S;
   volatile int* abort_flag = s_abort;
 
   if (warp == 0) {
@@ -225,7 +285,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       long long armed = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int t = u / S, sp = u - t * S;
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         int row0, row1;
         bool has1 = true;
@@ -239,7 +300,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const int nload = (ti.nrows + xb - 1) / xb;
         const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int kb0 = sp * nk / S, kb1 = (sp + 1) * nk / S;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -279,7 +341,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       const uint32_t fmt = p.fp8 ? 0u : 1u;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+        const int t = u / S, sp = u - t * S;
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
@@ -293,7 +356,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d1 = d0 + (uint32_t)p.tn;
         const int n_mma = ((ti.nrows + 15) / 16) * 16;
         const uint32_t idesc = umma_idesc(kWRows, n_mma, fmt);
-        for (int kb = 0; kb < nk; ++kb) {
+        const int kb0 = sp * nk / S, kb1 = (sp + 1) * nk / S;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(&full[stage], phase, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -305,7 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(xa + kk * 32);
-            const uint32_t accum = (kb | kk) != 0;
+            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
             if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             if (has1) {
@@ -338,79 +402,99 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int m = 32 * q + lane;
+    const size_t part_stride = (size_t)2 * p.tn * kWRows;   // floats per unit: [2][tn][128]
+    uint32_t ebar_parity = 0;
     int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+      const int t = u / S;
       const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
       const int acc = it % p.n_acc;
       const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
       if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * cols_per_acc);
+      // output features of this thread's accumulator row, and weight scales
+      int n0, n1;
+      bool has1 = true;
+      float s0 = 1.f, s1 = 1.f;
       if (p.gateup) {
-        const int n = ti.wt * kWRows + m;
-        float sg = 1.f, su = 1.f;
+        n0 = ti.wt * kWRows + m;
+        n1 = n0;
         if (p.fp8) {
-          sg = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n);
-          su = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n);
-        }
-        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
-        for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float g[16], u[16];
-          // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
-          const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-          tmem_ld16(tb + c, g);
-          tmem_ld16(tb + p.tn + c, u);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = c + i;
-            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-            if (j < ti.nrows) {
-              const int row = ti.r0 + j;
-              float gv = g[i], uv = u[i];
-              if (p.fp8) {
-                gv = gv * sa * sg;
-                uv = uv * sa * su;
-              }
-              const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
-              h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
-            }
-          }
+          s0 = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n0);
+          s1 = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n0);
         }
       } else {
-        const int n0 = ti.wt * 2 * kWRows + m;
-        const int n1 = n0 + kWRows;
-        const bool has1 = n1 < p.n_out;   // uniform across the warp (n_out % 128 == 0)
-        float sw0 = 1.f, sw1 = 1.f;
+        n0 = ti.wt * 2 * kWRows + m;
+        n1 = n0 + kWRows;
+        has1 = n1 < p.n_out;   // uniform across the warp (n_out % 128 == 0)
         if (p.fp8) {
-          sw0 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n0);
-          if (has1) sw1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
+          s0 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n0);
+          if (has1) s1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
         }
-        float* o = reinterpret_cast<float*>(p.out);
+      }
+      if (S == 1) {
         for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float v0[16], v1[16];
-          // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
-          const bool in = lane < 16 && c + lane < ti.nrows;
-          const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
-          const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-          tmem_ld16(tb + c, v0);
-          if (has1) tmem_ld16(tb + p.tn + c, v1);
+          float a0[16], a1[16];
+          tmem_ld16(tb + c, a0);
+          if (has1) tmem_ld16(tb + p.tn + c, a1);
+          if (p.gateup) epi_gateup(p, ti, c, n0, s0, s1, a0, a1, lane);
+          else epi_down(p, ti, c, n0, n1, has1, s0, s1, a0, a1, lane);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      } else {
+        // split K: store this unit's partial accumulators, release TMEM; the
+        // last unit of the tile to finish sums the partials in split order
+        float* mine = p.part + (size_t)u * part_stride;
+        for (int c = 16 * half; c < ti.nrows; c += 32) {
+          float a0[16], a1[16];
+          tmem_ld16(tb + c, a0);
+          if (has1) tmem_ld16(tb + p.tn + c, a1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int slot = __shfl_sync(0xffffffffu, slot_l, i);
-            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-            if (c + i < ti.nrows) {
-              if (slot < p.n_slots) {
-                float* yr = o + (long long)slot * p.n_out;
-                yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
-                if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
+            mine[(size_t)(c + i) * kWRows + m] = a0[i];
+            if (has1) mine[(size_t)(p.tn + c + i) * kWRows + m] = a1[i];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        __threadfence();
+        if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(p.tile_cnt + t, 1);
+          *s_last = old == S - 1;
+          if (old == S - 1) p.tile_cnt[t] = 0;   // ready for the next call
+        }
+        if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
+        if (*s_last) {
+          __threadfence();
+          const float* first = p.part + (size_t)t * S * part_stride;
+          for (int c = 16 * half; c < ti.nrows; c += 32) {
+            float a0[16], a1[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a0[i] = a1[i] = 0.f;
+            for (int sp = 0; sp < S; ++sp) {
+              const float* src = first + (size_t)sp * part_stride;
+              float b0[16], b1[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                b0[i] = __ldcg(src + (size_t)(c + i) * kWRows + m);
+                b1[i] = has1 ? __ldcg(src + (size_t)(p.tn + c + i) * kWRows + m) : 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                a0[i] += b0[i];
+                a1[i] += b1[i];
               }
             }
+            if (p.gateup) epi_gateup(p, ti, c, n0, s0, s1, a0, a1, lane);
+            else epi_down(p, ti, c, n0, n1, has1, s0, s1, a0, a1, lane);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
 
@@ -461,7 +545,7 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, long long
 size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
   const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
   (void)gateup;
-  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5) * 8 + 16 + (size_t)(4 * E + 1) * 4;
+  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 6) * 8 + 16 + (size_t)(4 * E + 1) * 4;
 }
 
 int gemm_pick_stages(int gateup, int tn, int E) {
