@@ -112,7 +112,7 @@ moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t*
 struct FfnShape {
   int T, H, I, E, k, bm, fp8, tn;
   long long P, NB, N;
-  int sp_gu, sp_dn;                 // K splits of the two GEMMs
+  int sk_gu, sk_dn;                 // stream-K for the two GEMMs (few tiles)
   long long tiles_gu, tiles_dn;     // upper bounds on the GEMMs' tile counts
 };
 
@@ -122,34 +122,13 @@ int device_sms() {
   return sms > 0 ? sms : 148;
 }
 
-// K splits for a GEMM with about est_tiles tiles of nk k-blocks: when the
-// tiles cannot fill the SMs several times over, split K so the last wave is
-// nearly full (each split keeps at least 4 k-blocks).
-int pick_splits(double est_tiles, int nk, int sms) {
-  if (est_tiles >= 4.0 * sms || est_tiles < 1) return 1;
-  int best = 1;
-  double best_score = -1;
-  const int max_s = nk / 4 < 16 ? nk / 4 : 16;
-  for (int sp = 1; sp <= (max_s > 1 ? max_s : 1); ++sp) {
-    const double units = est_tiles * sp;
-    const double waves = ceil(units / sms);
-    const double score = units / (waves * sms) - 0.01 * (sp - 1);
-    if (score > best_score + 1e-9) {
-      best_score = score;
-      best = sp;
-    }
-  }
-  return best;
-}
-
-int pick_tn(const FfnShape& s, int hint) {
-  if (hint) return hint;
-  const double avg = (double)s.N / s.E;  // slots per expert
-  long long need = (long long)((avg * 1.25 + s.bm - 1) / s.bm) * s.bm;
-  if (need < s.bm) need = s.bm;
-  int tn = 16;
-  while (tn < need && tn < 256) tn <<= 1;
-  return tn;
+// Stream-K when the tiles cannot fill the SMs several times over: a whole
+// number of tile waves would leave SMs idle in the last one.
+int pick_streamk(double est_tiles, int nk, int sms) {
+  if (nk < 2 || est_tiles < 1) return 0;
+  if (est_tiles >= 4.0 * sms) return 0;
+  const double waves = ceil(est_tiles / sms);
+  return est_tiles / (waves * sms) < 0.95 ? 1 : 0;
 }
 
 moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, int hint, FfnShape* s) {
@@ -178,8 +157,8 @@ moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, in
   const double groups = touched * ceil(padded / s->tn);
   const int eb = s->fp8 ? 1 : 2;
   const int sms = device_sms();
-  s->sp_gu = pick_splits(groups * (s->I / 128), s->H * eb / 128, sms);
-  s->sp_dn = pick_splits(groups * ((s->H + 255) / 256), s->I * eb / 128, sms);
+  s->sk_gu = pick_streamk(groups * (s->I / 128), s->H * eb / 128, sms);
+  s->sk_dn = pick_streamk(groups * ((s->H + 255) / 256), s->I * eb / 128, sms);
   return MOE_OK;
 }
 
@@ -198,11 +177,11 @@ FfnWs ffn_ws_layout(const FfnShape& s) {
   w.h = c.take((size_t)s.P * s.I * 2);
   w.hq = c.take(s.fp8 ? (size_t)s.P * s.I : 0);
   w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
-  const size_t unit = (size_t)2 * s.tn * 128 * sizeof(float);
-  w.part_gu = c.take(s.sp_gu > 1 ? (size_t)s.tiles_gu * s.sp_gu * unit : 0);
-  w.cnt_gu = c.take(s.sp_gu > 1 ? (size_t)s.tiles_gu * 4 : 0);
-  w.part_dn = c.take(s.sp_dn > 1 ? (size_t)s.tiles_dn * s.sp_dn * unit : 0);
-  w.cnt_dn = c.take(s.sp_dn > 1 ? (size_t)s.tiles_dn * 4 : 0);
+  const size_t unit = (size_t)6 * 2 * s.tn * 128 * sizeof(float);   // 6 contributors per tile at most
+  w.part_gu = c.take(s.sk_gu ? (size_t)s.tiles_gu * unit : 0);
+  w.cnt_gu = c.take(s.sk_gu ? (size_t)s.tiles_gu * 4 : 0);
+  w.part_dn = c.take(s.sk_dn ? (size_t)s.tiles_dn * unit : 0);
+  w.cnt_dn = c.take(s.sk_dn ? (size_t)s.tiles_dn * 4 : 0);
   w.total = c.off;
   return w;
 }
@@ -267,10 +246,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
-  g1.p.splits = s.sp_gu;
+  g1.p.streamk = s.sk_gu;
   g1.p.part = reinterpret_cast<float*>(ws + L.part_gu);
   g1.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_gu);
-  if (s.sp_gu > 1) MOE_CU(cudaMemsetAsync(g1.p.tile_cnt, 0, (size_t)s.tiles_gu * 4, stream));
+  if (s.sk_gu) MOE_CU(cudaMemsetAsync(g1.p.tile_cnt, 0, (size_t)s.tiles_gu * 4, stream));
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -298,10 +277,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
-  g2.p.splits = s.sp_dn;
+  g2.p.streamk = s.sk_dn;
   g2.p.part = reinterpret_cast<float*>(ws + L.part_dn);
   g2.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_dn);
-  if (s.sp_dn > 1) MOE_CU(cudaMemsetAsync(g2.p.tile_cnt, 0, (size_t)s.tiles_dn * 4, stream));
+  if (s.sk_dn) MOE_CU(cudaMemsetAsync(g2.p.tile_cnt, 0, (size_t)s.tiles_dn * 4, stream));
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));

@@ -36,6 +36,7 @@ constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilog
 constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
+constexpr int kMaxContrib = 6;   // stream-K contributors per tile (share >= nk/4 k-blocks)
 
 // Plan layout (int32), written by plan_kernel from the align&sort outputs.
 //   [0] tiles of the gate/up GEMM   [1] tiles of the down GEMM   [2] tn
@@ -152,6 +153,54 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
 // Token rows of the tile are loaded in boxes of x_box rows, only as many as
 // the token group has (rounded up to x_box).
 __device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
+
+// Work iteration.  Plain mode: whole tiles t = blockIdx.x, +gridDim.x, ...
+// Stream-K mode (few tiles): the n_tiles * nk k-blocks are cut into equal
+// contiguous shares, one per CTA, so every SM streams the same number of
+// weight bytes; a tile whose k-blocks span several CTAs has nc contributors,
+// this CTA being contributor ci (in k order).
+struct Seg {
+  int t, kb0, kb1, nc, ci;
+};
+struct SegIter {
+  long long pos, end, w;  // stream-K: current/end k-block of this CTA, share size
+  int u;                  // plain: next tile
+};
+__device__ __forceinline__ void seg_begin(SegIter& it, bool streamk, int n_tiles, int nk) {
+  if (streamk) {
+    const long long total = (long long)n_tiles * nk;
+    long long w = (total + gridDim.x - 1) / gridDim.x;
+    const long long wmin = (nk + 3) / 4;   // at most ~5 contributors per tile
+    it.w = w > wmin ? w : wmin;
+    it.pos = (long long)blockIdx.x * it.w;
+    it.end = it.pos + it.w < total ? it.pos + it.w : total;
+  } else {
+    it.u = blockIdx.x;
+  }
+}
+__device__ __forceinline__ bool seg_next(SegIter& it, bool streamk, int n_tiles, int nk, Seg& sg) {
+  if (!streamk) {
+    if (it.u >= n_tiles) return false;
+    sg.t = it.u;
+    sg.kb0 = 0;
+    sg.kb1 = nk;
+    sg.nc = 1;
+    sg.ci = 0;
+    it.u += gridDim.x;
+    return true;
+  }
+  if (it.pos >= it.end) return false;
+  sg.t = (int)(it.pos / nk);
+  sg.kb0 = (int)(it.pos - (long long)sg.t * nk);
+  const long long left = it.end - it.pos;
+  sg.kb1 = left < nk - sg.kb0 ? sg.kb0 + (int)left : nk;
+  const long long c_first = (long long)sg.t * nk / it.w;
+  const long long c_last = ((long long)(sg.t + 1) * nk - 1) / it.w;
+  sg.nc = (int)(c_last - c_first + 1);
+  sg.ci = (int)(blockIdx.x - c_first);
+  it.pos += sg.kb1 - sg.kb0;
+  return true;
+}
 
 // Final math of 16 token columns [c, c+16) of a gate/up tile for weight row
 // m of the tile (output feature n): h = bf16(silu(g*scale) * (u*scale)).
@@ -271,9 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
   const int cols_per_acc = 2 * p.tn;
   const int xb = x_box_rows(p.tn);
-  // work unit u = (tile u / S, K split u % S); splits of a tile are adjacent
-  const int S = p.splits;
-  const int n_units = n_tiles * S;
+  const bool streamk = p.streamk != 0;
   volatile int* abort_flag = s_abort;
 
   if (warp == 0) {
@@ -285,9 +332,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       long long armed = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int t = u / S, sp = u - t * S;
-        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      SegIter sit;
+      Seg sg;
+      seg_begin(sit, streamk, n_tiles, nk);
+      while (ok && seg_next(sit, streamk, n_tiles, nk, sg)) {
+        const TileInfo ti = decode_tile(sg.t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         int row0, row1;
         bool has1 = true;
         if (p.gateup) {
@@ -300,8 +349,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const int nload = (ti.nrows + xb - 1) / xb;
         const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
-        const int kb0 = sp * nk / S, kb1 = (sp + 1) * nk / S;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -341,9 +389,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       const uint32_t fmt = p.fp8 ? 0u : 1u;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-        const int t = u / S, sp = u - t * S;
-        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      SegIter sit;
+      Seg sg;
+      seg_begin(sit, streamk, n_tiles, nk);
+      for (; ok && seg_next(sit, streamk, n_tiles, nk, sg); ++it) {
+        const TileInfo ti = decode_tile(sg.t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
         const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
@@ -356,8 +406,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d1 = d0 + (uint32_t)p.tn;
         const int n_mma = ((ti.nrows + 15) / 16) * 16;
         const uint32_t idesc = umma_idesc(kWRows, n_mma, fmt);
-        const int kb0 = sp * nk / S, kb1 = (sp + 1) * nk / S;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!wait_or_abort(&full[stage], phase, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -369,7 +418,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(xa + kk * 32);
-            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
             if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             if (has1) {
@@ -402,11 +451,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int m = 32 * q + lane;
-    const size_t part_stride = (size_t)2 * p.tn * kWRows;   // floats per unit: [2][tn][128]
+    const size_t part_stride = (size_t)2 * p.tn * kWRows;   // floats per partial: [2][tn][128]
     uint32_t ebar_parity = 0;
     int it = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
-      const int t = u / S;
+    SegIter sit;
+    Seg sg;
+    seg_begin(sit, streamk, n_tiles, nk);
+    for (; seg_next(sit, streamk, n_tiles, nk, sg); ++it) {
+      const int t = sg.t;
       const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
       const int acc = it % p.n_acc;
       const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
@@ -433,7 +485,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (has1) s1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
         }
       }
-      if (S == 1) {
+      if (sg.nc == 1) {
         for (int c = 16 * half; c < ti.nrows; c += 32) {
           float a0[16], a1[16];
           tmem_ld16(tb + c, a0);
@@ -445,9 +497,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
       } else {
-        // split K: store this unit's partial accumulators, release TMEM; the
-        // last unit of the tile to finish sums the partials in split order
-        float* mine = p.part + (size_t)u * part_stride;
+        // the tile's k-blocks span several CTAs: store this contribution,
+        // release TMEM; the last contributor sums all of them in k order
+        float* mine = p.part + ((size_t)t * kMaxContrib + sg.ci) * part_stride;
         for (int c = 16 * half; c < ti.nrows; c += 32) {
           float a0[16], a1[16];
           tmem_ld16(tb + c, a0);
@@ -461,23 +513,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        __threadfence();
         if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
         if (threadIdx.x == 64) {
+          __threadfence();   // releases the whole epilogue's stores (ordered by the barrier)
           const int old = atomicAdd(p.tile_cnt + t, 1);
-          *s_last = old == S - 1;
-          if (old == S - 1) p.tile_cnt[t] = 0;   // ready for the next call
+          *s_last = old == sg.nc - 1;
+          if (old == sg.nc - 1) p.tile_cnt[t] = 0;   // ready for the next call
         }
         if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
         if (*s_last) {
           __threadfence();
-          const float* first = p.part + (size_t)t * S * part_stride;
+          const float* first = p.part + (size_t)t * kMaxContrib * part_stride;
           for (int c = 16 * half; c < ti.nrows; c += 32) {
             float a0[16], a1[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) a0[i] = a1[i] = 0.f;
-            for (int sp = 0; sp < S; ++sp) {
-              const float* src = first + (size_t)sp * part_stride;
+            for (int ci = 0; ci < sg.nc; ++ci) {
+              const float* src = first + (size_t)ci * part_stride;
               float b0[16], b1[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
