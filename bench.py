@@ -552,6 +552,8 @@ def run_only(args):
             cfg = cfg.with_(bm=int(p[2:]))
         elif p.startswith("T"):
             cfg = cfg.with_(T=int(p[1:]))
+        elif p.startswith("E"):
+            cfg = cfg.with_(E=int(p[1:]))
         elif p == "bias":
             cfg = cfg.with_(bias=True)
     rep, _, _ = layer_report(m, cfg, steps, warmup, dev, pk, parts[1])
@@ -567,7 +569,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--only", default=None,
-                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>] "
+                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>][_E<N>] "
                          "(configs: tiny, p5, deepseek, mixtral, decode) or align_<T>")
     args = ap.parse_args()
     if args.only:

@@ -40,6 +40,8 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
 
 def build(verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
+    if os.path.exists(LIB):
+        os.remove(LIB)   # never leave a stale library behind a failed build
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), SOURCES))
     cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC",

@@ -1,7 +1,6 @@
 // Host side of the C ABI declared in include/moe_b200.h: argument checks,
 // workspace carving and kernel launches.  No device memory is allocated and
 // no call synchronises the host.
-#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -112,23 +111,16 @@ moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t*
 struct FfnShape {
   int T, H, I, E, k, bm, fp8, tn;
   long long P, NB, N;
-  int sk_gu, sk_dn;                 // stream-K for the two GEMMs (few tiles)
-  long long tiles_gu, tiles_dn;     // upper bounds on the GEMMs' tile counts
 };
 
-int device_sms() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms > 0 ? sms : 148;
-}
-
-// Stream-K when the tiles cannot fill the SMs several times over: a whole
-// number of tile waves would leave SMs idle in the last one.
-int pick_streamk(double est_tiles, int nk, int sms) {
-  if (nk < 2 || est_tiles < 1) return 0;
-  if (est_tiles >= 4.0 * sms) return 0;
-  const double waves = ceil(est_tiles / sms);
-  return est_tiles / (waves * sms) < 0.95 ? 1 : 0;
+int pick_tn(const FfnShape& s, int hint) {
+  if (hint) return hint;
+  const double avg = (double)s.N / s.E;  // slots per expert
+  long long need = (long long)((avg * 1.25 + s.bm - 1) / s.bm) * s.bm;
+  if (need < s.bm) need = s.bm;
+  int tn = 16;
+  while (tn < need && tn < 256) tn <<= 1;
+  return tn;
 }
 
 moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, int hint, FfnShape* s) {
@@ -145,25 +137,11 @@ moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, in
   s->NB = (s->P + bm - 1) / bm;
   s->tn = pick_tn(*s, hint);
   if ((long long)s->P * (s->H > s->I ? s->H : s->I) >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
-  // tile-count bound: every touched expert pads by < bm rows and splits into tn-row groups
-  const long long touched_max = s->N < s->E ? s->N : s->E;
-  const long long groups_max = (s->N + s->tn - 1) / s->tn + touched_max * ((s->bm - 1 + s->tn - 1) / s->tn + 1);
-  s->tiles_gu = groups_max * (s->I / 128);
-  s->tiles_dn = groups_max * ((s->H + 255) / 256);
-  // expected tiles under uniform routing (one group per touched expert when tn covers it)
-  const double touched = s->E * (1.0 - pow(1.0 - 1.0 / s->E, (double)s->N));
-  const double rows = (double)s->N / (touched > 0 ? touched : 1);
-  const double padded = ceil(rows / s->bm) * s->bm;
-  const double groups = touched * ceil(padded / s->tn);
-  const int eb = s->fp8 ? 1 : 2;
-  const int sms = device_sms();
-  s->sk_gu = pick_streamk(groups * (s->I / 128), s->H * eb / 128, sms);
-  s->sk_dn = pick_streamk(groups * ((s->H + 255) / 256), s->I * eb / 128, sms);
   return MOE_OK;
 }
 
 struct FfnWs {
-  size_t plan, xq, sx, A, sA, h, hq, sH, part_gu, cnt_gu, part_dn, cnt_dn, total;
+  size_t plan, xq, sx, A, sA, h, hq, sH, total;
 };
 
 FfnWs ffn_ws_layout(const FfnShape& s) {
@@ -177,11 +155,6 @@ FfnWs ffn_ws_layout(const FfnShape& s) {
   w.h = c.take((size_t)s.P * s.I * 2);
   w.hq = c.take(s.fp8 ? (size_t)s.P * s.I : 0);
   w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
-  const size_t unit = (size_t)6 * 2 * s.tn * 128 * sizeof(float);   // 6 contributors per tile at most
-  w.part_gu = c.take(s.sk_gu ? (size_t)s.tiles_gu * unit : 0);
-  w.cnt_gu = c.take(s.sk_gu ? (size_t)s.tiles_gu * 4 : 0);
-  w.part_dn = c.take(s.sk_dn ? (size_t)s.tiles_dn * unit : 0);
-  w.cnt_dn = c.take(s.sk_dn ? (size_t)s.tiles_dn * 4 : 0);
   w.total = c.off;
   return w;
 }
@@ -246,10 +219,6 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
-  g1.p.streamk = s.sk_gu;
-  g1.p.part = reinterpret_cast<float*>(ws + L.part_gu);
-  g1.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_gu);
-  if (s.sk_gu) MOE_CU(cudaMemsetAsync(g1.p.tile_cnt, 0, (size_t)s.tiles_gu * 4, stream));
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -277,10 +246,6 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
-  g2.p.streamk = s.sk_dn;
-  g2.p.part = reinterpret_cast<float*>(ws + L.part_dn);
-  g2.p.tile_cnt = reinterpret_cast<int*>(ws + L.cnt_dn);
-  if (s.sk_dn) MOE_CU(cudaMemsetAsync(g2.p.tile_cnt, 0, (size_t)s.tiles_dn * 4, stream));
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));

@@ -36,7 +36,6 @@ constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilog
 constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
-constexpr int kMaxContrib = 6;   // stream-K contributors per tile (share >= nk/4 k-blocks)
 
 // Plan layout (int32), written by plan_kernel from the align&sort outputs.
 //   [0] tiles of the gate/up GEMM   [1] tiles of the down GEMM   [2] tn
@@ -154,108 +153,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
 // the token group has (rounded up to x_box).
 __device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
 
-// Work iteration.  Plain mode: whole tiles t = blockIdx.x, +gridDim.x, ...
-// Stream-K mode (few tiles): the n_tiles * nk k-blocks are cut into equal
-// contiguous shares, one per CTA, so every SM streams the same number of
-// weight bytes; a tile whose k-blocks span several CTAs has nc contributors,
-// this CTA being contributor ci (in k order).
-struct Seg {
-  int t, kb0, kb1, nc, ci;
-};
-struct SegIter {
-  long long pos, end, w;  // stream-K: current/end k-block of this CTA, share size
-  int u;                  // plain: next tile
-};
-__device__ __forceinline__ void seg_begin(SegIter& it, bool streamk, int n_tiles, int nk) {
-  if (streamk) {
-    const long long total = (long long)n_tiles * nk;
-    long long w = (total + gridDim.x - 1) / gridDim.x;
-    const long long wmin = (nk + 3) / 4;   // at most ~5 contributors per tile
-    it.w = w > wmin ? w : wmin;
-    it.pos = (long long)blockIdx.x * it.w;
-    it.end = it.pos + it.w < total ? it.pos + it.w : total;
-  } else {
-    it.u = blockIdx.x;
-  }
-}
-__device__ __forceinline__ bool seg_next(SegIter& it, bool streamk, int n_tiles, int nk, Seg& sg) {
-  if (!streamk) {
-    if (it.u >= n_tiles) return false;
-    sg.t = it.u;
-    sg.kb0 = 0;
-    sg.kb1 = nk;
-    sg.nc = 1;
-    sg.ci = 0;
-    it.u += gridDim.x;
-    return true;
-  }
-  if (it.pos >= it.end) return false;
-  sg.t = (int)(it.pos / nk);
-  sg.kb0 = (int)(it.pos - (long long)sg.t * nk);
-  const long long left = it.end - it.pos;
-  sg.kb1 = left < nk - sg.kb0 ? sg.kb0 + (int)left : nk;
-  const long long c_first = (long long)sg.t * nk / it.w;
-  const long long c_last = ((long long)(sg.t + 1) * nk - 1) / it.w;
-  sg.nc = (int)(c_last - c_first + 1);
-  sg.ci = (int)(blockIdx.x - c_first);
-  it.pos += sg.kb1 - sg.kb0;
-  return true;
-}
-
-// Final math of 16 token columns [c, c+16) of a gate/up tile for weight row
-// m of the tile (output feature n): h = bf16(silu(g*scale) * (u*scale)).
-__device__ __forceinline__ void epi_gateup(const GemmParams& p, const TileInfo& ti, int c, int n, float sg, float su,
-                                           const float (&g)[16], const float (&u)[16], int lane) {
-  // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
-  const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-    if (c + i < ti.nrows) {
-      float gv = g[i], uv = u[i];
-      if (p.fp8) {
-        gv = gv * sa * sg;
-        uv = uv * sa * su;
-      }
-      const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
-      h[(long long)(ti.r0 + c + i) * p.n_out + n] = __float2bfloat16_rn(hv);
-    }
-  }
-}
-
-// Final math of 16 token columns of a down tile: y[slot, n0|n1] = acc * scales.
-__device__ __forceinline__ void epi_down(const GemmParams& p, const TileInfo& ti, int c, int n0, int n1, bool has1,
-                                         float sw0, float sw1, const float (&v0)[16], const float (&v1)[16],
-                                         int lane) {
-  // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
-  const bool in = lane < 16 && c + lane < ti.nrows;
-  const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
-  const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-  float* o = reinterpret_cast<float*>(p.out);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int slot = __shfl_sync(0xffffffffu, slot_l, i);
-    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-    if (c + i < ti.nrows && slot < p.n_slots) {
-      float* yr = o + (long long)slot * p.n_out;
-      yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
-      if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
-    }
-  }
-}
-
-// Barrier of the eight epilogue warps on an mbarrier (8 arrivals), bounded
-// like every other wait; `parity` alternates per use.
-__device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& parity, long long timeout_ns,
-                                         volatile int* abort_flag, int lane) {
-  __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
-  const bool ok = wait_or_abort(bar, parity, timeout_ns, abort_flag);
-  parity ^= 1u;
-  return ok;
-}
-
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         GemmParams p) {
@@ -272,10 +169,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = bars + 2 * p.stages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* ebar = drain + 1;   // epilogue-warp barrier (split K)
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ebar + 1);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  int* s_last = s_abort + 1;
   int* s_start = s_abort + 3;   // keep 16-byte alignment of the arrays below
   int* s_rows = s_start + E;
   int* s_groups = s_rows + E;
@@ -293,7 +188,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
-    mbar_init(ebar, 8);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
@@ -320,7 +214,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
   const int cols_per_acc = 2 * p.tn;
   const int xb = x_box_rows(p.tn);
-  const bool streamk = p.streamk != 0;
   volatile int* abort_flag = s_abort;
 
   if (warp == 0) {
@@ -332,11 +225,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       long long armed = 0;
       bool ok = true;
-      SegIter sit;
-      Seg sg;
-      seg_begin(sit, streamk, n_tiles, nk);
-      while (ok && seg_next(sit, streamk, n_tiles, nk, sg)) {
-        const TileInfo ti = decode_tile(sg.t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         int row0, row1;
         bool has1 = true;
         if (p.gateup) {
@@ -349,7 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const int nload = (ti.nrows + xb - 1) / xb;
         const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -389,11 +279,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       const uint32_t fmt = p.fp8 ? 0u : 1u;
-      SegIter sit;
-      Seg sg;
-      seg_begin(sit, streamk, n_tiles, nk);
-      for (; ok && seg_next(sit, streamk, n_tiles, nk, sg); ++it) {
-        const TileInfo ti = decode_tile(sg.t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
         const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
@@ -406,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d1 = d0 + (uint32_t)p.tn;
         const int n_mma = ((ti.nrows + 15) / 16) * 16;
         const uint32_t idesc = umma_idesc(kWRows, n_mma, fmt);
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {
           if (!wait_or_abort(&full[stage], phase, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
@@ -418,7 +305,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(xa + kk * 32);
-            const uint32_t accum = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb | kk) != 0;
             if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
             if (has1) {
@@ -451,102 +338,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int m = 32 * q + lane;
-    const size_t part_stride = (size_t)2 * p.tn * kWRows;   // floats per partial: [2][tn][128]
-    uint32_t ebar_parity = 0;
     int it = 0;
-    SegIter sit;
-    Seg sg;
-    seg_begin(sit, streamk, n_tiles, nk);
-    for (; seg_next(sit, streamk, n_tiles, nk, sg); ++it) {
-      const int t = sg.t;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
       const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
       const int acc = it % p.n_acc;
       const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
       if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * cols_per_acc);
-      // output features of this thread's accumulator row, and weight scales
-      int n0, n1;
-      bool has1 = true;
-      float s0 = 1.f, s1 = 1.f;
       if (p.gateup) {
-        n0 = ti.wt * kWRows + m;
-        n1 = n0;
+        const int n = ti.wt * kWRows + m;
+        float sg = 1.f, su = 1.f;
         if (p.fp8) {
-          s0 = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n0);
-          s1 = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n0);
+          sg = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + n);
+          su = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + n);
         }
-      } else {
-        n0 = ti.wt * 2 * kWRows + m;
-        n1 = n0 + kWRows;
-        has1 = n1 < p.n_out;   // uniform across the warp (n_out % 128 == 0)
-        if (p.fp8) {
-          s0 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n0);
-          if (has1) s1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
-        }
-      }
-      if (sg.nc == 1) {
+        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
         for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float a0[16], a1[16];
-          tmem_ld16(tb + c, a0);
-          if (has1) tmem_ld16(tb + p.tn + c, a1);
-          if (p.gateup) epi_gateup(p, ti, c, n0, s0, s1, a0, a1, lane);
-          else epi_down(p, ti, c, n0, n1, has1, s0, s1, a0, a1, lane);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      } else {
-        // the tile's k-blocks span several CTAs: store this contribution,
-        // release TMEM; the last contributor sums all of them in k order
-        float* mine = p.part + ((size_t)t * kMaxContrib + sg.ci) * part_stride;
-        for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float a0[16], a1[16];
-          tmem_ld16(tb + c, a0);
-          if (has1) tmem_ld16(tb + p.tn + c, a1);
+          float g[16], u[16];
+          // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
+          const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
+          tmem_ld16(tb + c, g);
+          tmem_ld16(tb + p.tn + c, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            mine[(size_t)(c + i) * kWRows + m] = a0[i];
-            if (has1) mine[(size_t)(p.tn + c + i) * kWRows + m] = a1[i];
+            const int j = c + i;
+            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
+            if (j < ti.nrows) {
+              const int row = ti.r0 + j;
+              float gv = g[i], uv = u[i];
+              if (p.fp8) {
+                gv = gv * sa * sg;
+                uv = uv * sa * su;
+              }
+              const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
+              h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
+            }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
-        if (threadIdx.x == 64) {
-          __threadfence();   // releases the whole epilogue's stores (ordered by the barrier)
-          const int old = atomicAdd(p.tile_cnt + t, 1);
-          *s_last = old == sg.nc - 1;
-          if (old == sg.nc - 1) p.tile_cnt[t] = 0;   // ready for the next call
+      } else {
+        const int n0 = ti.wt * 2 * kWRows + m;
+        const int n1 = n0 + kWRows;
+        const bool has1 = n1 < p.n_out;   // uniform across the warp (n_out % 128 == 0)
+        float sw0 = 1.f, sw1 = 1.f;
+        if (p.fp8) {
+          sw0 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n0);
+          if (has1) sw1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
         }
-        if (!epi_sync(ebar, ebar_parity, p.timeout_ns, abort_flag, lane)) break;
-        if (*s_last) {
-          __threadfence();
-          const float* first = p.part + (size_t)t * kMaxContrib * part_stride;
-          for (int c = 16 * half; c < ti.nrows; c += 32) {
-            float a0[16], a1[16];
+        float* o = reinterpret_cast<float*>(p.out);
+        for (int c = 16 * half; c < ti.nrows; c += 32) {
+          float v0[16], v1[16];
+          // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
+          const bool in = lane < 16 && c + lane < ti.nrows;
+          const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
+          const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
+          tmem_ld16(tb + c, v0);
+          if (has1) tmem_ld16(tb + p.tn + c, v1);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) a0[i] = a1[i] = 0.f;
-            for (int ci = 0; ci < sg.nc; ++ci) {
-              const float* src = first + (size_t)ci * part_stride;
-              float b0[16], b1[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                b0[i] = __ldcg(src + (size_t)(c + i) * kWRows + m);
-                b1[i] = has1 ? __ldcg(src + (size_t)(p.tn + c + i) * kWRows + m) : 0.f;
-              }
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                a0[i] += b0[i];
-                a1[i] += b1[i];
+          for (int i = 0; i < 16; ++i) {
+            const int slot = __shfl_sync(0xffffffffu, slot_l, i);
+            const float sa = __shfl_sync(0xffffffffu, sa_l, i);
+            if (c + i < ti.nrows) {
+              if (slot < p.n_slots) {
+                float* yr = o + (long long)slot * p.n_out;
+                yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
+                if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
               }
             }
-            if (p.gateup) epi_gateup(p, ti, c, n0, s0, s1, a0, a1, lane);
-            else epi_down(p, ti, c, n0, n1, has1, s0, s1, a0, a1, lane);
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
 
@@ -597,7 +461,7 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, long long
 size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
   const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
   (void)gateup;
-  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 6) * 8 + 16 + (size_t)(4 * E + 1) * 4;
+  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5) * 8 + 16 + (size_t)(4 * E + 1) * 4;
 }
 
 int gemm_pick_stages(int gateup, int tn, int E) {

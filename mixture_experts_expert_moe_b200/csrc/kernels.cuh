@@ -80,9 +80,6 @@ struct GemmParams {
   void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] (one row per slot)
   int32_t* status;
   long long timeout_ns;
-  int streamk;           // 1: equal k-block shares per CTA (few tiles); partials below
-  float* part;           // [tiles][6][2][tn][128] fp32 partial accumulators (stream-K)
-  int* tile_cnt;         // per-tile arrival counters, zero on entry (stream-K)
 };
 
 struct GemmLaunch {
