@@ -97,18 +97,44 @@ __device__ int block_exclusive_scan(int* a, int n) {
   return s_total;
 }
 
-// Loads kSub sub-steps (32 consecutive slots each) of a warp's sub-chunk;
-// ids outside [0, E) and slots past the end become -1.  All loads are issued
-// before any value is used (a use right after a load would expose every load
-// latency in turn).  Plain (L2) loads: in the fused routing kernel the ids
-// were written earlier in the same launch.
-__device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, long long end, int lane, int E,
-                                          int (&key)[kSub]) {
+// Issues the loads of kSub sub-steps (32 consecutive slots each) of a warp's
+// sub-chunk without using the values, so they can be in flight while the
+// previous sub-steps are processed.  Plain (L2) loads: in the fused routing
+// kernel the ids were written earlier in the same launch.
+__device__ __forceinline__ void load_raw(const int32_t* ids, long long base, long long end, int lane,
+                                         int (&key)[kSub]) {
 #pragma unroll
   for (int q = 0; q < kSub; ++q) {
     const long long i = base + q * 32 + lane;
     key[q] = i < end ? __ldcg(ids + i) : -1;
   }
+}
+
+// Lanes of the warp holding the same value v in [0, 2^kBits): one ballot per
+// bit, all independent, so they issue back to back.
+template <int kBits>
+__device__ __forceinline__ unsigned match_peers(int v) {
+  unsigned ones[kBits];
+#pragma unroll
+  for (int b = 0; b < kBits; ++b) ones[b] = __ballot_sync(0xffffffffu, (v >> b) & 1);
+  unsigned peers = 0xffffffffu;
+#pragma unroll
+  for (int b = 0; b < kBits; ++b) peers &= ((v >> b) & 1) ? ones[b] : ~ones[b];
+  return peers;
+}
+
+template <int N>
+struct Log2 {
+  static constexpr int value = 1 + Log2<N / 2>::value;
+};
+template <>
+struct Log2<1> {
+  static constexpr int value = 0;
+};
+
+// ids outside [0, E) and slots past the end become -1; returns whether an id
+// was out of range.
+__device__ __forceinline__ bool validate_keys(long long base, long long end, int lane, int E, int (&key)[kSub]) {
   bool bad = false;
 #pragma unroll
   for (int q = 0; q < kSub; ++q) {
@@ -121,8 +147,9 @@ __device__ __forceinline__ bool load_keys(const int32_t* ids, long long base, lo
   return bad;
 }
 
-// kGate: the CTA first gates the tokens whose slots it owns (its chunk is a
-// multiple of k) and writes ids/weights.  kPlan: CTA 0 finally writes the
+// EPL = ceil(E/32) rounded up to a power of two (the gating's logits per lane
+// and the width of the id matching).  kGate: the CTA first gates the tokens
+// whose slots it owns (its chunk is a multiple of k) and writes ids/weights.  kPlan: CTA 0 finally writes the
 // grouped GEMMs' tile plan from the padded offsets.  With one CTA there is no
 // grid-wide wait.
 template <int EPL, bool kGate, bool kPlan>
@@ -156,13 +183,20 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   int* my = wcnt + warp * E;
 
   // ---- (D) count: each warp into its own row (shared-memory atomics) -----
+  // the next step's ids are loaded while the current ones are counted
   bool bad = false;
-  for (long long base = w_begin; base < w_end; base += 32 * kSub) {
-    int key[kSub];
-    bad |= load_keys(p.ids, base, w_end, lane, E, key);
+  {
+    int key[kSub], nxt[kSub];
+    if (w_begin < w_end) load_raw(p.ids, w_begin, w_end, lane, key);
+    for (long long base = w_begin; base < w_end; base += 32 * kSub) {
+      if (base + 32 * kSub < w_end) load_raw(p.ids, base + 32 * kSub, w_end, lane, nxt);
+      bad |= validate_keys(base, w_end, lane, E, key);
 #pragma unroll
-    for (int q = 0; q < kSub; ++q)
-      if (key[q] >= 0) atomicAdd(&my[key[q]], 1);
+      for (int q = 0; q < kSub; ++q)
+        if (key[q] >= 0) atomicAdd(&my[key[q]], 1);
+#pragma unroll
+      for (int q = 0; q < kSub; ++q) key[q] = nxt[q];
+    }
   }
   if (bad) s_bad = 1;
   __syncthreads();
@@ -237,41 +271,51 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   const int bpc = (nblk + G - 1) / G;
   const int j0 = blockIdx.x * bpc;
   const int j1 = min(nblk, j0 + bpc);
-  for (int j = j0 + warp; j < j1; j += kAlignWarps) {   // one warp per block
+  for (int j = j0 + tid; j < j1; j += blockDim.x) {   // one thread per block
     const int pos = j * p.bm;
     int lo = 0, hi = E - 1;  // last expert whose segment starts at or before pos
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
     }
-    if (lane == 0) p.expert_ids[j] = lo;
-    const int fill = s_off[lo] + s_tot[lo];  // first padding position of expert lo
-    for (int q = max(fill, pos) + lane; q < pos + p.bm; q += 32) p.sorted[q] = p.N;
+    p.expert_ids[j] = lo;
+  }
+  // padding (only in an expert's last block): the part inside this CTA's blocks
+  for (int e = warp; e < E; e += kAlignWarps) {
+    const int beg = max(s_off[e] + s_tot[e], j0 * p.bm);
+    const int end = min(s_off[e] + (s_tot[e] + p.bm - 1) / p.bm * p.bm, j1 * p.bm);
+    for (int q = beg + lane; q < end; q += 32) p.sorted[q] = p.N;
   }
 
   // ---- (P) stable placement ------------------------------------------------
-  // The shared-memory rank chain needs a warp barrier per sub-step; the global
-  // stores are issued after the chain so those barriers do not wait on them.
-  for (long long base = w_begin; base < w_end; base += 32 * kSub) {
-    int key[kSub], dest[kSub];
-    load_keys(p.ids, base, w_end, lane, E, key);
+  // Ranks: the lowest lane of each group of equal ids takes the group's
+  // positions with one shared-memory atomicAdd on the warp's row (it returns
+  // the running count) and shares it by a shuffle.  The warp's atomics reach
+  // its row in issue order, so equal ids keep the order of the sub-steps.
+  {
+    int key[kSub], nxt[kSub];
+    if (w_begin < w_end) load_raw(p.ids, w_begin, w_end, lane, key);
+    for (long long base = w_begin; base < w_end; base += 32 * kSub) {
+      if (base + 32 * kSub < w_end) load_raw(p.ids, base + 32 * kSub, w_end, lane, nxt);
+      validate_keys(base, w_end, lane, E, key);
+      int dest[kSub];
 #pragma unroll
-    for (int q = 0; q < kSub; ++q) {
-      const int kq = key[q];
-      const unsigned peers = __match_any_sync(0xffffffffu, kq);
-      const int cnt = kq >= 0 ? my[kq] : 0;
-      __syncwarp();
-      dest[q] = -1;
-      if (kq >= 0) {
-        const unsigned below = peers & lanemask_lt();
-        dest[q] = s_base[kq] + cnt + __popc(below);
-        if (below == 0) my[kq] = cnt + __popc(peers);
+      for (int q = 0; q < kSub; ++q) {
+        const int kq = key[q];
+        // ids + 1 are in [0, 32*EPL]: Log2<32*EPL> + 1 bits (-1, no slot, becomes 0)
+        const unsigned peers = match_peers<Log2<32 * EPL>::value + 1>(kq + 1);
+        const int leader = __ffs(peers) - 1;
+        int old = 0;
+        if (kq >= 0 && lane == leader) old = atomicAdd(&my[kq], __popc(peers));
+        old = __shfl_sync(0xffffffffu, old, leader);
+        dest[q] = kq >= 0 ? s_base[kq] + old + __popc(peers & lanemask_lt()) : -1;
       }
-      __syncwarp();
-    }
 #pragma unroll
-    for (int q = 0; q < kSub; ++q)
-      if (dest[q] >= 0) p.sorted[dest[q]] = (int)(base + q * 32 + lane);
+      for (int q = 0; q < kSub; ++q)
+        if (dest[q] >= 0) p.sorted[dest[q]] = (int)(base + q * 32 + lane);
+#pragma unroll
+      for (int q = 0; q < kSub; ++q) key[q] = nxt[q];
+    }
   }
 
   if (kPlan && blockIdx.x == 0) {
@@ -329,7 +373,13 @@ static cudaError_t launch_route_impl(K kernel, const AlignParams& p, const Route
 
 cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream) {
   RouteExtra r = {};
-  return launch_route_impl(route_kernel<1, false, false>, p, r, grid, stream);
+  const int epl = (p.E + 31) / 32;
+  if (epl <= 1) return launch_route_impl(route_kernel<1, false, false>, p, r, grid, stream);
+  if (epl <= 2) return launch_route_impl(route_kernel<2, false, false>, p, r, grid, stream);
+  if (epl <= 4) return launch_route_impl(route_kernel<4, false, false>, p, r, grid, stream);
+  if (epl <= 8) return launch_route_impl(route_kernel<8, false, false>, p, r, grid, stream);
+  if (epl <= 16) return launch_route_impl(route_kernel<16, false, false>, p, r, grid, stream);
+  return launch_route_impl(route_kernel<32, false, false>, p, r, grid, stream);
 }
 
 cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream) {

@@ -114,3 +114,16 @@ def test_grid_wait_times_out_cleanly(cuda_device):
     ids = align_ids(64, 8, 2, seed=1, dist="uniform")
     s, b, n, st2 = _run_align(ids, 8, 16, cuda_device)
     assert st2 == 0 and n == oracle.align_sort(ids, 8, 16)[2]
+
+
+@pytest.mark.parametrize("T,k,E,dist", [(200000, 1, 3, "uniform"), (60000, 2, 8, "zipf"), (30000, 4, 5, "zipf")])
+def test_align_sort_stable_under_heavy_collisions(cuda_device, T, k, E, dist):
+    """Many equal ids per warp step: the stable order inside every segment must
+    match the oracle on every one of several runs."""
+    ids = align_ids(T, E, k, seed=T + E, dist=dist)
+    ref_s, ref_b, ref_n = oracle.align_sort(ids, E, 32)
+    for _ in range(4):
+        s, b, n, st = _run_align(ids, E, 32, cuda_device)
+        assert st == 0 and n == ref_n
+        np.testing.assert_array_equal(s[:n], ref_s)
+        np.testing.assert_array_equal(b[:n // 32], ref_b)
