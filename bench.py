@@ -119,12 +119,13 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_layer(m, cfg, dev, out_dtype=torch.bfloat16):
+def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0):
     d = make_layer(cfg, device=dev)
     if cfg.a8w8:
-        layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype)
+        layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype,
+                           tile_tokens=tile_tokens)
     else:
-        layer = m.MoELayer(d["w13"], d["w2"], cfg.k, cfg.bm, out_dtype=out_dtype)
+        layer = m.MoELayer(d["w13"], d["w2"], cfg.k, cfg.bm, out_dtype=out_dtype, tile_tokens=tile_tokens)
     return d, layer
 
 
@@ -245,8 +246,8 @@ def traffic_for(kernel, workload):
     return None
 
 
-def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False):
-    d, layer = build_layer(m, cfg, dev)
+def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile_tokens=0):
+    d, layer = build_layer(m, cfg, dev, tile_tokens=tile_tokens)
     touched, _ = touched_experts(layer, d)
     ms_eager, st = time_layer(m, cfg, layer, d, steps, warmup)
     ms_graph = time_graph(m, cfg, layer, d, steps, warmup)
@@ -547,6 +548,7 @@ def run_only(args):
         print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
         return
     cfg = CONFIGS[parts[0]].with_(a8w8=parts[1] == "a8w8")
+    tile = 0
     for p in parts[2:]:
         if p.startswith("bm"):
             cfg = cfg.with_(bm=int(p[2:]))
@@ -554,9 +556,11 @@ def run_only(args):
             cfg = cfg.with_(T=int(p[1:]))
         elif p.startswith("E"):
             cfg = cfg.with_(E=int(p[1:]))
+        elif p.startswith("tn"):
+            tile = int(p[2:])
         elif p == "bias":
             cfg = cfg.with_(bias=True)
-    rep, _, _ = layer_report(m, cfg, steps, warmup, dev, pk, parts[1])
+    rep, _, _ = layer_report(m, cfg, steps, warmup, dev, pk, parts[1], tile_tokens=tile)
     print(json.dumps(rep))
 
 
@@ -569,7 +573,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--only", default=None,
-                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>][_E<N>] "
+                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>][_E<N>][_tn<N>] "
                          "(configs: tiny, p5, deepseek, mixtral, decode) or align_<T>")
     args = ap.parse_args()
     if args.only:
