@@ -219,6 +219,8 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
+  // many tokens per expert (256-token tiles): the GEMMs are tensor-bound, use SM pairs
+  g1.p.pair = s.tn == 256;
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -246,6 +248,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g2.p.pair = s.tn == 256;
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));

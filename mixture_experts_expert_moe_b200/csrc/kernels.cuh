@@ -80,6 +80,7 @@ struct GemmParams {
   void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] (one row per slot)
   int32_t* status;
   long long timeout_ns;
+  int pair;              // 1: two-SM (cluster of 2) kernel, M = 256 per tile pair, tn = 256
 };
 
 struct GemmLaunch {
