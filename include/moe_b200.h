@@ -252,6 +252,16 @@ MOE_API moe_status_t moe_forward(const moe_forward_args* args, void* ws, size_t 
 MOE_API moe_status_t moe_test_wait_timeout(void* ws, int32_t* dev_status, long long timeout_ns,
                                    void* stream);
 
+/* moe_test_quant_division checks the E4M3 quantiser's quotient path (one
+ * reciprocal per row plus a fused-multiply-add correction per element) against
+ * an IEEE fp32 division for every pair of bf16 values (v, amax) with
+ * 0 < amax <= the largest finite bf16 and |v| <= amax: it compares the E4M3
+ * codes of v / s, s = amax / 448.  ws: at least 32 bytes of device memory,
+ * cleared by the call; on completion of the stream it holds uint64 pairs
+ * checked, uint64 mismatches and uint32 (v bits << 16 | amax bits) of one
+ * mismatch (0 if none).  Test hook; the method's pages have no counterpart. */
+MOE_API moe_status_t moe_test_quant_division(void* ws, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

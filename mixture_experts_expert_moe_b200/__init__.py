@@ -24,7 +24,7 @@ EXPORTED = [
     "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
     "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
     "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
-    "moe_align_sort_noalloc",
+    "moe_align_sort_noalloc", "moe_test_quant_division",
 ]
 
 _vp = ctypes.c_void_p
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_forward": (_i, [ctypes.POINTER(ForwardArgs), _vp, ctypes.c_size_t, _vp, _vp]),
             "moe_test_wait_timeout": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
             "moe_align_sort_noalloc": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+            "moe_test_quant_division": (_i, [_vp, _vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -290,3 +291,15 @@ def run_wait_timeout_check(timeout_ns: int, device="cuda"):
            "moe_test_wait_timeout")
     torch.cuda.synchronize()
     return int(st.item())
+
+
+def run_quant_division_check(device="cuda"):
+    """Exhaustive check of the E4M3 quantiser's quotient path against IEEE
+    division over all bf16 pairs (v, amax), |v| <= amax.  Returns
+    (pairs checked, mismatches, one failing (v bits << 16 | amax bits))."""
+    lib = load_library()
+    ws = torch.zeros(4, dtype=torch.int64, device=device)
+    _check(lib.moe_test_quant_division(_ptr(ws), _stream(torch.device(device))), "moe_test_quant_division")
+    torch.cuda.synchronize()
+    c = ws.cpu().tolist()
+    return c[0], c[1], c[2] & 0xFFFFFFFF

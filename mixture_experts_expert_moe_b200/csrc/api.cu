@@ -219,8 +219,6 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
-  // many tokens per expert (256-token tiles): the GEMMs are tensor-bound, use SM pairs
-  g1.p.pair = s.tn == 256;
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -248,7 +246,6 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
-  g2.p.pair = s.tn == 256;
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
@@ -483,6 +480,17 @@ moe_status_t moe_test_wait_timeout(void* ws, int32_t* dev_status, long long time
   cudaStream_t cs = (cudaStream_t)stream;
   MOE_CU(cudaMemsetAsync(ws, 0, sizeof(int), cs));
   MOE_CU(moe::launch_wait_timeout(static_cast<int*>(ws), dev_status, timeout_ns, cs));
+  return MOE_OK;
+}
+
+moe_status_t moe_test_quant_division(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  MOE_CU(cudaMemsetAsync(ws, 0, 32, cs));
+  unsigned long long* counts = static_cast<unsigned long long*>(ws);
+  MOE_CU(moe::launch_quant_division_check(counts, reinterpret_cast<unsigned int*>(counts + 2), cs));
   return MOE_OK;
 }
 

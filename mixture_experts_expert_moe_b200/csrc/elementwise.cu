@@ -83,20 +83,56 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 // ---------------------------------------------------------------------------
 // Per-row E4M3 quantisation (aiter issue 1248: per-token FP8 activations;
 // GC-MoE: requantisation between the GEMMs).  s = amax / 448 in fp32 (1 for
-// an all-zero row); code = e4m3_rne_satfinite(v / s) with an IEEE fp32
-// division.  One warp per row with the row held in registers (VPL 16-byte
-// vectors of 8 bf16 per lane); rows longer than 16*32*8 take two passes.  With
-// a row map the kernel also gathers (sorted row r quantises its token).
+// an all-zero row); code = e4m3_rne_satfinite(v / s) with v / s the correctly
+// rounded fp32 quotient.  One warp per row with the row held in registers (VPL
+// 16-byte vectors of 8 bf16 per lane); longer rows take one CTA per row (up
+// to 256*16*8 elements), beyond that two passes.  With a row map the kernel also gathers (sorted row r quantises its
+// token).
+//
+// The quotient comes from one reciprocal per row and a correction step per
+// element (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990): with r = RN(1/s)
+// and q = RN(v r), the residual v - q s is exact under a fused multiply-add and
+// RN(q + residual * r) = RN(v / s).  The residual is exact only while it does
+// not underflow: for s >= 2^-90 that holds for every quotient of magnitude
+// >= 2^-11, and smaller quotients all encode to a signed zero (their sign is
+// carried over from q, since the sum can turn -0 into +0).  Rows with a
+// smaller scale divide element by element.  moe_test_quant_division
+// checks the resulting codes against a per-element IEEE division for every
+// pair of bf16 values (v, amax) with |v| <= amax.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t e4m3_pack4(float a, float b, float c, float d) {
-  const uint32_t qa = __nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qb = __nv_cvt_float_to_fp8(b, __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qc = __nv_cvt_float_to_fp8(c, __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qd = __nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3);
-  return qa | (qb << 8) | (qc << 16) | (qd << 24);
+struct RowScale {
+  float s;     // the row's scale
+  float r;     // RN(1 / s) when the correction step applies, else 0
+};
+
+__device__ __forceinline__ RowScale row_scale(float amax) {
+  RowScale rs;
+  rs.s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  rs.r = rs.s >= 0x1p-90f ? __frcp_rn(rs.s) : 0.f;
+  return rs;
+}
+
+// RN(v / s): correction step (kFast, needs rs.r != 0) or IEEE division
+template <bool kFast>
+__device__ __forceinline__ float div_by_scale(float v, const RowScale& rs) {
+  if (!kFast) return __fdiv_rn(v, rs.s);
+  const float q = v * rs.r;
+  const float res = fmaf(-q, rs.s, v);
+  return copysignf(fmaf(res, rs.r, q), q);
+}
+
+// two quotients -> two E4M3 codes (a in the low byte)
+__device__ __forceinline__ uint32_t e4m3_pack2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+template <bool kFast>
+__device__ __forceinline__ uint32_t quant_pair(uint32_t u, const RowScale& rs) {
+  return e4m3_pack2(div_by_scale<kFast>(bf16_lo(u), rs), div_by_scale<kFast>(bf16_hi(u), rs));
 }
 
 __device__ __forceinline__ float absmax8(const uint4& v) {
@@ -104,13 +140,27 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
                fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
 }
 
-__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
+template <bool kFast>
+__device__ __forceinline__ uint2 quant8(const uint4& v, const RowScale& rs) {
   uint2 o;
-  o.x = e4m3_pack4(__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s), __fdiv_rn(bf16_lo(v.y), s),
-                   __fdiv_rn(bf16_hi(v.y), s));
-  o.y = e4m3_pack4(__fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s), __fdiv_rn(bf16_lo(v.w), s),
-                   __fdiv_rn(bf16_hi(v.w), s));
+  o.x = quant_pair<kFast>(v.x, rs) | (quant_pair<kFast>(v.y, rs) << 16);
+  o.y = quant_pair<kFast>(v.z, rs) | (quant_pair<kFast>(v.w, rs) << 16);
   return o;
+}
+
+// the row's codes from n register-resident vectors v[i] -> dst[c0 + stride*i]
+template <int V>
+__device__ __forceinline__ void quant_store(const uint4 (&v)[V], const RowScale& rs, uint2* dst, int c0, int stride,
+                                            int vec) {
+  if (rs.r != 0.f) {
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+      if (c0 + stride * i < vec) dst[c0 + stride * i] = quant8<true>(v[i], rs);
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+      if (c0 + stride * i < vec) dst[c0 + stride * i] = quant8<false>(v[i], rs);
+  }
 }
 
 // gather (optional): row r quantises token sorted[r] / k of src (padding
@@ -149,17 +199,57 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int c = lane + 32 * i;
-      if (c < vec) dst[c] = quant8(v[i], s);
-    }
-    if (lane == 0) scale[r] = s;
+    const RowScale rs = row_scale(amax);
+    quant_store<VPL>(v, rs, dst, lane, 32, vec);
+    if (lane == 0) scale[r] = rs.s;
   }
 }
 
-// Rows longer than the register-resident limit: one warp per row, two passes
+// Long rows (up to 256*16*8 elements): one CTA of 256 threads per row, the row
+// held in registers (VPT 16-byte vectors per thread), a block-wide amax, one
+// read of the row.
+template <int VPT>
+__global__ void __launch_bounds__(256) quant_rows_block_kernel(const uint4* __restrict__ src,
+                                                               const int32_t* __restrict__ sorted, int N, int k,
+                                                               const int32_t* __restrict__ nrows_dev, int nrows,
+                                                               int vec, uint2* __restrict__ q,
+                                                               float* __restrict__ scale) {
+  __shared__ float s_amax[8];
+  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = blockIdx.x; r < n; r += gridDim.x) {
+    const long long sr = quant_src_row(sorted, r, N, k);
+    uint2* dst = q + (long long)r * vec;
+    if (sr < 0) {
+      for (int c = threadIdx.x; c < vec; c += 256) dst[c] = make_uint2(0, 0);
+      if (threadIdx.x == 0) scale[r] = 1.f;
+      continue;
+    }
+    const uint4* row = src + sr * vec;
+    uint4 v[VPT];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + 256 * i;
+      v[i] = c < vec ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
+      amax = fmaxf(amax, absmax8(v[i]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) s_amax[warp] = amax;
+    __syncthreads();
+    amax = s_amax[lane & 7];
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    __syncthreads();   // s_amax is rewritten by the next row
+    const RowScale rs = row_scale(amax);
+    quant_store<VPT>(v, rs, dst, threadIdx.x, 256, vec);
+    if (threadIdx.x == 0) scale[r] = rs.s;
+  }
+}
+
+// Rows longer than the register-resident limits: one warp per row, two passes
+
 // (the second pass re-reads the row from L1/L2).
 __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __restrict__ src,
                                                                const int32_t* __restrict__ sorted, int N, int k,
@@ -182,9 +272,12 @@ __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __re
     for (int c = lane; c < vec; c += 32) amax = fmaxf(amax, absmax8(__ldg(row + c)));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    for (int c = lane; c < vec; c += 32) dst[c] = quant8(__ldg(row + c), s);
-    if (lane == 0) scale[r] = s;
+    const RowScale rs = row_scale(amax);
+    if (rs.r != 0.f)
+      for (int c = lane; c < vec; c += 32) dst[c] = quant8<true>(__ldg(row + c), rs);
+    else
+      for (int c = lane; c < vec; c += 32) dst[c] = quant8<false>(__ldg(row + c), rs);
+    if (lane == 0) scale[r] = rs.s;
   }
 }
 
@@ -223,8 +316,53 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int
   else if (vpl <= 4) MOE_QUANT(4);
   else if (vpl <= 8) MOE_QUANT(8);
   else if (vpl <= 16) MOE_QUANT(16);
-  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
+  else {
+    const int vpt = (vec + 255) / 256;
+    const long long cap = (long long)sm_count() * 8;
+    const int gb = (int)(nrows < 1 ? 1 : (nrows < cap ? nrows : cap));
+#define MOE_QUANT_B(V) quant_rows_block_kernel<V><<<gb, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale)
+    if (vpt <= 4) MOE_QUANT_B(4);
+    else if (vpt <= 8) MOE_QUANT_B(8);
+    else if (vpt <= 16) MOE_QUANT_B(16);
+    else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
+#undef MOE_QUANT_B
+  }
 #undef MOE_QUANT
+  return cudaGetLastError();
+}
+
+// Exhaustive check of the quotient path: block b takes amax = the positive
+// bf16 with bit pattern b + 1 (up to the largest finite, 0x7F7F) and every
+// bf16 v with |v| <= amax, both signs; the codes of quant_pair must equal
+// e4m3(__fdiv_rn(v, s)).  counts[0] += pairs checked, counts[1] += mismatches;
+// first_bad keeps one failing (v bits << 16 | amax bits).
+__global__ void __launch_bounds__(256) quant_division_check_kernel(unsigned long long* counts,
+                                                                   unsigned int* first_bad) {
+  const uint32_t amax_bits = blockIdx.x + 1;
+  const float amax = __uint_as_float(amax_bits << 16);
+  const RowScale rs = row_scale(amax);
+  unsigned long long bad = 0;
+  for (uint32_t vb = threadIdx.x; vb <= amax_bits; vb += blockDim.x) {
+    const uint32_t pos = vb, neg = vb | 0x8000u;
+    const uint32_t packed = pos | (neg << 16);
+    const uint32_t got = rs.r != 0.f ? quant_pair<true>(packed, rs) : quant_pair<false>(packed, rs);
+    const uint32_t want = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(pos << 16), rs.s), __NV_SATFINITE,
+                                                          __NV_E4M3) |
+                          ((uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(__uint_as_float(neg << 16), rs.s),
+                                                           __NV_SATFINITE, __NV_E4M3)
+                           << 8);
+    if (got != want) {
+      ++bad;
+      atomicCAS(first_bad, 0u, (vb << 16) | amax_bits);
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, off);
+  if ((threadIdx.x & 31) == 0 && bad) atomicAdd(counts + 1, bad);
+  if (threadIdx.x == 0) atomicAdd(counts, 2ull * (amax_bits + 1));
+}
+
+cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s) {
+  quant_division_check_kernel<<<0x7F7F, 256, 0, s>>>(counts, first_bad);
   return cudaGetLastError();
 }
 

@@ -239,6 +239,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const int nload = (ti.nrows + xb - 1) / xb;
         const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
+        // weights streamed once (one token group) go first; re-read ones stay in L2
+        const uint64_t pol_wt = s_groups[ti.e] > 1 ? pol_x : pol_w;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
             ok = false;
@@ -247,8 +249,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sb = smem + (size_t)stage * stage_bytes;
           mbar_arrive_expect_tx(&full[stage], tx);
           const int kc = kb * k_elems;
-          tma_load_2d(sb, &tm_w, &full[stage], kc, row0, pol_w);
-          if (has1) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, row1, pol_w);
+          tma_load_2d(sb, &tm_w, &full[stage], kc, row0, pol_wt);
+          if (has1) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, row1, pol_wt);
           for (int l = 0; l < nload; ++l)
             tma_load_2d(sb + w_bytes + l * xb * kStageK, &tm_x, &full[stage], kc, ti.r0 + l * xb, pol_x);
           ++armed;
@@ -423,291 +425,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Two-SM variant for compute-bound shapes (many tokens per expert): a CTA pair
-// (cluster of 2) computes a 256-weight-row x tn-token tile with
-// tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own 128 weight rows
-// and half of the token rows, so per-SM shared-memory traffic per MMA is half
-// of the one-SM kernel's (which is bound by shared-memory bandwidth at tn = 256).
-//   gate/up: CTA r holds gate rows [f0, f0+64) and up rows [f0, f0+64) of the
-//            same 64 features (f0 = wt*128 + 64r); its accumulator lanes 0..63
-//            are gate, 64..127 up; the epilogue pairs them through shared memory.
-//   down:    CTA r holds output rows [wt*256 + 128r, +128).
-// The even CTA issues the MMAs; TMA loads of both CTAs complete on its full
-// barriers; commits arrive on both CTAs' barriers; the odd CTA's epilogue
-// releases the accumulator on the even CTA's barrier.  No multicast loads.
-// ---------------------------------------------------------------------------
-// Final math of 16 token columns [c, c+16) of a gate/up tile for output
-// feature n: h = bf16(silu(g * scale) * (u * scale)).
-__device__ __forceinline__ void epi_gateup(const GemmParams& p, const TileInfo& ti, int c, int n, float sg, float su,
-                                           const float (&g)[16], const float (&u)[16], int lane) {
-  // lanes 0..15 fetch the chunk's row scales; shuffles broadcast them
-  const float sa_l = (p.fp8 && lane < 16 && c + lane < ti.nrows) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-    if (c + i < ti.nrows) {
-      float gv = g[i], uv = u[i];
-      if (p.fp8) {
-        gv = gv * sa * sg;
-        uv = uv * sa * su;
-      }
-      const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
-      h[(long long)(ti.r0 + c + i) * p.n_out + n] = __float2bfloat16_rn(hv);
-    }
-  }
-}
-
-// Final math of 16 token columns of a down tile: y[slot, n0 (and n1)] = acc * scales.
-__device__ __forceinline__ void epi_down(const GemmParams& p, const TileInfo& ti, int c, int n0, int n1, bool has1,
-                                         float sw0, float sw1, const float (&v0)[16], const float (&v1)[16],
-                                         int lane) {
-  // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
-  const bool in = lane < 16 && c + lane < ti.nrows;
-  const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
-  const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-  float* o = reinterpret_cast<float*>(p.out);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int slot = __shfl_sync(0xffffffffu, slot_l, i);
-    const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-    if (c + i < ti.nrows && slot < p.n_slots) {
-      float* yr = o + (long long)slot * p.n_out;
-      yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
-      if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
-    }
-  }
-}
-
-constexpr int kPairXch = 2 * 2 * 16 * 32;   // floats: [half][quarter pair][16 cols][32 lanes]
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                             GemmParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int E = p.E;
-  const int half_tn = p.tn / 2;                        // token rows this CTA stages
-  const int stage_bytes = kWTileBytes + half_tn * kStageK;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
-  uint64_t* full = bars;                  // used on the even CTA only
-  uint64_t* empty = bars + p.stages;
-  uint64_t* acc_full = bars + 2 * p.stages;
-  uint64_t* acc_empty = acc_full + 2;     // used on the even CTA only (16 arrivals)
-  uint64_t* spare = acc_empty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(spare + 2);
-  int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  int* s_start = s_abort + 3;
-  int* s_rows = s_start + E;
-  int* s_groups = s_rows + E;
-  int* s_pref = s_groups + E;   // E + 1
-  float* xch = reinterpret_cast<float*>(s_pref + E + 1 + 3);   // 16-byte aligned below
-  xch = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(xch) + 15) & ~uintptr_t(15));
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-
-  if (warp == 0 && lane == 0) {
-    for (int s = 0; s < p.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 16);
-    }
-    *s_abort = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_x);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(s_tmem, p.tmem_cols);
-    tmem_relinquish_pair();
-  }
-  const int pref_off = p.gateup ? 4 + 3 * E : 5 + 4 * E;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) {
-    s_start[i] = p.plan[4 + i];
-    s_rows[i] = p.plan[4 + E + i];
-    s_groups[i] = p.plan[4 + 2 * E + i];
-  }
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_pref[i] = p.plan[pref_off + i];
-  const int n_tiles = p.plan[p.gateup ? 0 : 1];
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();   // the even CTA's barriers exist before the odd CTA signals them
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
-
-  const int nk = p.K * (p.fp8 ? 1 : 2) / kStageK;
-  const int k_elems = p.fp8 ? kStageK : kStageK / 2;
-  const int xb = 32;
-  const int nload = half_tn / xb;
-  volatile int* abort_flag = s_abort;
-  // shared::cluster addresses of the even CTA's barriers
-  const uint32_t full0 = mapa_shared(smem_u32(full), 0);
-  const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
-
-  if (warp == 0) {
-    // ---------------- TMA producer (both CTAs) ----------------
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      const uint32_t tx_pair = 2u * (uint32_t)stage_bytes;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
-        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
-        int ra, rb;   // first weight row of the two 64-row boxes (gate/up) or of the 128-row box (down)
-        if (p.gateup) {
-          ra = ti.e * 2 * p.n_out + ti.wt * kWRows + (int)rank * 64;
-          rb = ra + p.n_out;
-        } else {
-          ra = ti.e * p.n_out + ti.wt * 2 * kWRows + (int)rank * kWRows;
-          rb = 0;
-        }
-        const int xr = ti.r0 + (int)rank * half_tn;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = smem + (size_t)stage * stage_bytes;
-          const uint32_t fb = full0 + (uint32_t)(stage * 8);
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx_pair);
-          const int kc = kb * k_elems;
-          if (p.gateup) {
-            tma_load_2d_pair(sb, &tm_w, fb, kc, ra, pol_w);                   // gate rows -> rows 0..63
-            tma_load_2d_pair(sb + kWTileBytes / 2, &tm_w, fb, kc, rb, pol_w);  // up rows -> rows 64..127
-          } else {
-            tma_load_2d_pair(sb, &tm_w, fb, kc, ra, pol_w);
-          }
-          for (int l = 0; l < nload; ++l)
-            tma_load_2d_pair(sb + kWTileBytes + l * xb * kStageK, &tm_x, fb, kc, xr + l * xb, pol_x);
-          if (++stage == p.stages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      // drain: every stage's last commit has landed before the CTA may exit
-      for (int i = 0; i < p.stages && ok; ++i) {
-        if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) break;
-        if (++stage == p.stages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (even CTA) ----------------
-    if (lane == 0 && rank == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      bool ok = true;
-      const uint32_t fmt = p.fp8 ? 0u : 1u;
-      const uint32_t idesc = umma_idesc(2 * kWRows, p.tn, fmt);
-      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
-        if (!wait_or_abort(&acc_empty[acc], acc_phase ^ 1, p.timeout_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)(acc * p.tn);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_or_abort(&full[stage], phase, p.timeout_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t w0 = smem_u32(smem + (size_t)stage * stage_bytes);
-          const uint32_t xa = w0 + (uint32_t)kWTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kStageK / 32; ++kk) {
-            const uint32_t accum = (kb | kk) != 0;
-            if (p.fp8) mma_e4m3_pair(d, umma_desc_sw128(w0 + kk * 32), umma_desc_sw128(xa + kk * 32), idesc, accum);
-            else mma_bf16_pair(d, umma_desc_sw128(w0 + kk * 32), umma_desc_sw128(xa + kk * 32), idesc, accum);
-          }
-          tc_commit_pair(&empty[stage]);
-          if (++stage == p.stages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
-        tc_commit_pair(&acc_full[acc]);
-      }
-    }
-  } else {
-    // ---------------- epilogue: warps 2..9 of both CTAs ----------------
-    const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int m = 32 * q + lane;   // accumulator row (TMEM lane) of this thread
-    int it = 0;
-    for (int t = pair; t < n_tiles; t += n_pairs, ++it) {
-      const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
-      const int acc = it & 1;
-      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
-      if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * p.tn);
-      if (p.gateup) {
-        // lanes 0..63 gate, 64..127 up of features f0 + (m & 63)
-        const int f = ti.wt * kWRows + (int)rank * 64 + (m & 63);
-        float sg = 1.f, su = 1.f;
-        if (p.fp8) {
-          sg = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + f);
-          su = __ldg(p.w_scale + (long long)ti.e * 2 * p.n_out + p.n_out + f);
-        }
-        float* xb2 = xch + ((half * 2 + (q & 1)) * 16) * 32;
-        const int bar_id = 1 + half * 2 + (q & 1);
-        for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float v[16];
-          tmem_ld16(tb + c, v);
-          if (q >= 2) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) xb2[i * 32 + lane] = v[i];
-          }
-          named_bar_sync(bar_id, 64);
-          if (q < 2) {
-            float u[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) u[i] = xb2[i * 32 + lane];
-            epi_gateup(p, ti, c, f, sg, su, v, u, lane);
-          }
-          named_bar_sync(bar_id, 64);
-        }
-      } else {
-        const int n = ti.wt * 2 * kWRows + (int)rank * kWRows + m;
-        const bool valid = n < p.n_out;   // uniform across the warp (n_out % 128 == 0)
-        const float sw = (p.fp8 && valid) ? __ldg(p.w_scale + (long long)ti.e * p.n_out + n) : 1.f;
-        for (int c = 16 * half; c < ti.nrows; c += 32) {
-          float v[16];
-          tmem_ld16(tb + c, v);
-          if (valid) epi_down(p, ti, c, n, n, false, sw, sw, v, v, lane);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty0 + (uint32_t)(acc * 8));
-    }
-  }
-
-  __syncthreads();
-  cluster_sync_all();   // neither CTA leaves while the other may still signal it
-  if (threadIdx.x == 0 && *abort_flag) dev_flag(p.status, MOE_DEV_TIMEOUT);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, p.tmem_cols);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -755,53 +472,7 @@ int gemm_pick_stages(int gateup, int tn, int E) {
   return s;
 }
 
-static size_t pair_smem_bytes(int tn, int stages, int E) {
-  const int stage_bytes = kWTileBytes + (tn / 2) * kStageK;
-  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 6) * 8 + 16 + (size_t)(4 * E + 4) * 4 + 16 +
-         (size_t)kPairXch * 4;
-}
-
-static int pair_pick_stages(int tn, int E) {
-  int s = 8;
-  while (s > 2 && pair_smem_bytes(tn, s, E) > 225 * 1024) --s;
-  return s;
-}
-
-static int launch_pair(GemmLaunch& L, cudaStream_t stream) {
-  GemmParams& p = L.p;
-  const int eb = p.fp8 ? 1 : 2;
-  CUtensorMap tw, tx;
-  if (!make_map(&tw, L.w, L.w_rows, p.K, eb, p.gateup ? 64 : kWRows)) return -1;
-  if (!make_map(&tx, L.x, L.x_rows, p.K, eb, 32)) return -1;
-  p.stages = pair_pick_stages(p.tn, p.E);
-  p.n_acc = 2;
-  int alloc = 32;
-  while (alloc < 2 * p.tn) alloc <<= 1;
-  p.tmem_cols = alloc;
-  const size_t smem = pair_smem_bytes(p.tn, p.stages, p.E);
-  cudaError_t e =
-      cudaFuncSetAttribute(grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return (int)e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(sms & ~1));
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return (int)cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, tw, tx, p);
-}
-
 int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream) {
-  if (L.p.pair) return launch_pair(L, stream);
   GemmParams& p = L.p;
   const int eb = p.fp8 ? 1 : 2;
   CUtensorMap tw, tx;

@@ -50,6 +50,7 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
 // sorted[r] / k (zero codes, scale 1 for padding slots >= N).
 cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
                               int nrows, int C, void* q, float* scale, cudaStream_t s);
+cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
 
@@ -80,7 +81,6 @@ struct GemmParams {
   void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] (one row per slot)
   int32_t* status;
   long long timeout_ns;
-  int pair;              // 1: two-SM (cluster of 2) kernel, M = 256 per tile pair, tn = 256
 };
 
 struct GemmLaunch {

@@ -23,8 +23,8 @@ SMALL = [
     MoEConfig("skew", T=257, H=256, I=128, E=32, k=8, bm=16, bias=True, seed=103),
     # few tokens per expert
     MoEConfig("fewtok", T=3, H=1024, I=512, E=16, k=2, bm=16, seed=104),
-    # many tokens per expert: 256-token tiles on SM pairs (two-SM MMA)
-    MoEConfig("pair", T=1024, H=512, I=384, E=4, k=2, bm=64, seed=105),
+    # many tokens per expert: 256-token tiles, several tiles per expert
+    MoEConfig("manytok", T=1024, H=512, I=384, E=4, k=2, bm=64, seed=105),
 ]
 
 
