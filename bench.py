@@ -137,8 +137,16 @@ def touched_experts(layer, d):
 
 
 def kernels_per_step(cfg, out_dtype):
-    n = 7                                         # gate, align, plan, gather, gate/up, down, combine
-    return n + (1 if cfg.a8w8 else 0)             # + requant
+    """Kernels of this library one moe_forward launches: the routing kernel
+    (gate + align + plan), the gather, the gate/up and down GEMMs and the
+    combine; a8w8 adds the requantisation, and above 4096 slots it
+    quantises each token once before the gather instead of inside it.  (The
+    memset of the routing kernel's grid-wait counter is a runtime call, not a
+    kernel of this library.)"""
+    n = 5
+    if cfg.a8w8:
+        n += 1 + (1 if cfg.T * cfg.k > 4096 else 0)
+    return n
 
 
 def time_layer(m, cfg, layer, d, steps, warmup, stage_times=True):
