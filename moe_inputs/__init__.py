@@ -20,6 +20,8 @@ inter 2048 shape):
 * router logits: ``x @ Wr`` with Wr ~ N(0, 0.02) in fp32 for the tiny
   layer, i.i.d. N(0, 1) otherwise (so the top-k set is a uniformly random
   k-subset); the skewed variant adds a per-expert N(0, 1) bias;
+* shared experts (DeepSeek-V3 has one) are drawn like the routed ones and
+  stored after them in the same weight tensors;
 * align-only ids: k distinct experts per token drawn one after another
   without replacement from Zipf(s) popularity over a seeded permutation of
   the experts (Gumbel-top-k, which has exactly that law), or uniformly.
@@ -50,6 +52,8 @@ class MoEConfig:
     bias: bool = False
     router: str = "normal"      # "normal": logits ~ N(0,1); "linear": x @ Wr
     seed: int = SEED_BASE
+    n_shared: int = 0           # always-on shared experts stored after the E routed ones
+    bias_mode: str = "logits"   # "logits": bias feeds selection and weights; "select": selection only
 
     def with_(self, **kw) -> "MoEConfig":
         return replace(self, **kw)
@@ -67,6 +71,10 @@ CONFIGS = {
                           seed=SEED_BASE + 3),
     # the aiter a8w8 issue's shape: 32 local experts, ~64 tokens each
     "p5": MoEConfig("p5", T=256, H=7168, I=2048, E=32, k=8, bm=64, seed=SEED_BASE + 5),
+    # DeepSeek-V3-shaped layer with its shared expert and the selection-only
+    # gating bias (aux-loss-free balancing)
+    "deepseek_shared": MoEConfig("deepseek_shared", T=2048, H=7168, I=2048, E=256, k=8, bm=64,
+                                 bias=True, n_shared=1, bias_mode="select", seed=SEED_BASE + 6),
     # decode sweep, FP8 a8w8 (T in 1, 16, 64, 256)
     "decode": MoEConfig("decode", T=64, H=7168, I=2048, E=256, k=8, bm=16,
                         a8w8=True, seed=SEED_BASE + 4),
@@ -106,9 +114,11 @@ def make_layer(cfg: MoEConfig, device="cpu", weights=True):
 
     Returns a dict with x (bf16 [T,H]), logits (f32 [T,E]), bias (f32 [E] or
     None) and, when ``weights``: w13/w2 (bf16) or w13_q/w13_s/w2_q/w2_s
-    (float8_e4m3fn codes + f32 scales).
+    (float8_e4m3fn codes + f32 scales) for the E routed experts followed by
+    the cfg.n_shared shared ones.
     """
     T, H, I, E = cfg.T, cfg.H, cfg.I, cfg.E
+    EW = E + cfg.n_shared
     s = cfg.seed
     d = {}
     d["x"] = normal((T, H), 1.0, s * 16 + 1, device, torch.bfloat16)
@@ -120,11 +130,11 @@ def make_layer(cfg: MoEConfig, device="cpu", weights=True):
     d["bias"] = normal((E,), 1.0, s * 16 + 4, device) if cfg.bias else None
     if weights:
         if cfg.a8w8:
-            d["w13_q"], d["w13_s"] = fp8_weights(E, 2 * I, H, 0.02, s * 16 + 5, device)
-            d["w2_q"], d["w2_s"] = fp8_weights(E, H, I, 0.02, s * 16 + 6, device)
+            d["w13_q"], d["w13_s"] = fp8_weights(EW, 2 * I, H, 0.02, s * 16 + 5, device)
+            d["w2_q"], d["w2_s"] = fp8_weights(EW, H, I, 0.02, s * 16 + 6, device)
         else:
-            d["w13"] = normal((E, 2 * I, H), 0.02, s * 16 + 5, device, torch.bfloat16)
-            d["w2"] = normal((E, H, I), 0.02, s * 16 + 6, device, torch.bfloat16)
+            d["w13"] = normal((EW, 2 * I, H), 0.02, s * 16 + 5, device, torch.bfloat16)
+            d["w2"] = normal((EW, H, I), 0.02, s * 16 + 6, device, torch.bfloat16)
     return d
 
 

@@ -19,6 +19,7 @@ from .moe_oracle import (  # noqa: F401
     e4m3_encode,
     e4m3_values,
     topk_gate,
+    add_shared,
     align_sort,
     quant_rows_e4m3,
     ffn_bf16,

@@ -28,8 +28,11 @@ Readings where the pages are silent (each is listed in the design doc):
 
 1. Top-k ties go to the lower expert index; ids are listed by descending
    logit.  Weights are the softmax over all E logits, renormalised over the
-   k selected ones.  A bias, when given, is added to the logits in fp32
-   before both selection and softmax.
+   k selected ones.  A bias, when given, is added to the logits in fp32,
+   either before both selection and softmax ("logits") or for the selection
+   only ("select", the weights then use the raw logits).
+1a. Shared experts have the routed experts' shape, see every token and enter
+   the combine with weight 1; they are stored after the routed experts.
 2. Within an expert's segment, slots keep ascending flat order
    (slot = t*k + j), as a counting sort gives.  Padding entries hold the
    sentinel T*k.  Experts with no slot get zero blocks.
@@ -134,28 +137,48 @@ def e4m3_encode(v) -> np.ndarray:
 #     opening definition: Top-K gating scores, with a gating bias in DSv3)
 # ---------------------------------------------------------------------------
 
-def topk_gate(logits, k: int, bias=None):
+def topk_gate(logits, k: int, bias=None, bias_mode: str = "logits"):
     """Top-k softmax gating.
 
     logits: float32 [T, E]; bias: float32 [E] or None (added in fp32).
-    Returns ids int32 [T, k] (descending logit, ties to the lower index) and
+    Returns ids int32 [T, k] (descending score, ties to the lower index) and
     weights float32 [T, k] = softmax(l)[sel] / sum(softmax(l)[sel]).
+
+    bias_mode "logits": the biased logits are both the selection score and
+    the l of the weights.  "select" ([AS] opening: DeepSeek's gating bias for
+    auxiliary-loss-free balancing): the biased logits only pick the experts;
+    the weights use the raw logits.
     """
+    if bias_mode not in ("logits", "select"):
+        raise ValueError(bias_mode)
     l32 = np.asarray(logits, dtype=np.float32)
+    score = l32
     if bias is not None:
-        l32 = (l32 + np.asarray(bias, dtype=np.float32)[None, :]).astype(np.float32)
+        score = (l32 + np.asarray(bias, dtype=np.float32)[None, :]).astype(np.float32)
     T, E = l32.shape
     if not (1 <= k <= E):
         raise ValueError("need 1 <= k <= E")
-    # stable sort of the negated logits keeps equal values in index order
-    order = np.argsort(-l32, axis=1, kind="stable")
+    # stable sort of the negated scores keeps equal values in index order
+    order = np.argsort(-score, axis=1, kind="stable")
     ids = order[:, :k].astype(np.int32)
-    l = l32.astype(np.float64)
+    l = (score if bias_mode == "logits" else l32).astype(np.float64)
     p = np.exp(l - l.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
     psel = np.take_along_axis(p, ids.astype(np.int64), axis=1)
     w = psel / psel.sum(axis=1, keepdims=True)
     return ids, w.astype(np.float32)
+
+
+def add_shared(ids, w, E: int, n_shared: int):
+    """Append the always-on shared experts ([AS] opening: DeepSeek's shared
+    expert, one of them) to every token's routing: experts E..E+n_shared-1,
+    weight 1 each, after the k routed choices."""
+    ids = np.asarray(ids, dtype=np.int32)
+    w = np.asarray(w, dtype=np.float32)
+    T = ids.shape[0]
+    sid = np.broadcast_to(E + np.arange(n_shared, dtype=np.int32), (T, n_shared))
+    return (np.concatenate([ids, sid], axis=1),
+            np.concatenate([w, np.ones((T, n_shared), np.float32)], axis=1))
 
 
 # ---------------------------------------------------------------------------
@@ -309,17 +332,21 @@ def combine(y, w):
 # ---------------------------------------------------------------------------
 
 def moe_forward(x, logits, k, w13, w2, bias=None, a8w8=False, w13_s=None,
-                w2_s=None, tokens=None):
+                w2_s=None, tokens=None, n_shared=0, bias_mode="logits"):
     """Gate -> (align, which only reorders) -> expert FFN -> combine.
 
-    Returns (out float64 [len(tokens) or T, H], ids, weights).  ``tokens``
-    restricts the FFN and combine to a subset of tokens (routing is computed
-    for all of them).
+    The weights hold E = logits.shape[1] routed experts followed by
+    ``n_shared`` shared experts; every token also goes to each shared expert
+    with weight 1.  Returns (out float64 [len(tokens) or T, H], ids, weights)
+    with ids/weights [T, k + n_shared].  ``tokens`` restricts the FFN and
+    combine to a subset of tokens (routing is computed for all of them).
     """
-    ids, w = topk_gate(logits, k, bias)
-    T = ids.shape[0]
+    ids, w = topk_gate(logits, k, bias, bias_mode)
+    if n_shared:
+        ids, w = add_shared(ids, w, np.asarray(logits).shape[1], n_shared)
+    T, kk = ids.shape
     toks = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
-    slots = (toks[:, None] * k + np.arange(k)[None, :]).reshape(-1)
+    slots = (toks[:, None] * kk + np.arange(kk)[None, :]).reshape(-1)
     if a8w8:
         y = ffn_a8w8(x, ids, w13, w13_s, w2, w2_s, slots=slots)
     else:

@@ -9,6 +9,8 @@
 * permuting tokens permutes the output; relabelling experts (weights and
   logit columns together) leaves it unchanged;
 * the combine is the weighted sum written with a library einsum-free loop;
+* shared experts add their dense FFN with weight 1 (the layer with them minus
+  the layer without them; routed outputs forced to zero);
 * a planted mistake (gate and up swapped) fails the dense pin.
 """
 import numpy as np
@@ -86,6 +88,46 @@ def test_forced_single_expert_is_dense():
     out, ids, w = mo.moe_forward(x, logits, 1, w13, w2)
     assert np.all(ids == 2) and np.all(w == 1.0)
     np.testing.assert_allclose(out, _dense_swiglu_bf16(x, w13[2], w2[2]), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("a8w8", [False, True])
+def test_shared_expert_adds_its_dense_ffn(a8w8):
+    """Shared experts enter with weight 1 for every token: the layer with
+    n_shared = 2 minus the same layer without them is the sum of the two
+    shared experts' dense FFNs (torch float64 matmuls)."""
+    cfg = MoEConfig("t", T=24, H=64, I=32, E=4, k=2, bm=8, a8w8=a8w8, n_shared=2, seed=17)
+    d = make_layer(cfg)
+    x, logits = to_numpy(d["x"]), to_numpy(d["logits"])
+    E = cfg.E
+    if a8w8:
+        w13q, w13s, w2q, w2s = (to_numpy(d[n]) for n in ("w13_q", "w13_s", "w2_q", "w2_s"))
+        out2, ids, w = mo.moe_forward(x, logits, cfg.k, w13q, w2q, a8w8=True, w13_s=w13s, w2_s=w2s,
+                                      n_shared=2)
+        out0, _, _ = mo.moe_forward(x, logits, cfg.k, w13q[:E], w2q[:E], a8w8=True, w13_s=w13s[:E],
+                                    w2_s=w2s[:E])
+        dense = sum(_dense_swiglu_a8w8(x, w13q[e], w13s[e], w2q[e], w2s[e]) for e in (E, E + 1))
+    else:
+        w13, w2 = to_numpy(d["w13"]), to_numpy(d["w2"])
+        out2, ids, w = mo.moe_forward(x, logits, cfg.k, w13, w2, n_shared=2)
+        out0, _, _ = mo.moe_forward(x, logits, cfg.k, w13[:E], w2[:E])
+        dense = sum(_dense_swiglu_bf16(x, w13[e], w2[e]) for e in (E, E + 1))
+    assert ids.shape == (cfg.T, cfg.k + 2)
+    np.testing.assert_array_equal(ids[:, cfg.k:], np.broadcast_to([E, E + 1], (cfg.T, 2)))
+    np.testing.assert_array_equal(w[:, cfg.k:], 1.0)
+    np.testing.assert_allclose(out2 - out0, dense, rtol=1e-5, atol=1e-6)
+
+
+def test_shared_expert_alone_when_routed_outputs_vanish():
+    """With every routed expert's down projection zero, the layer is the
+    shared expert's dense FFN whatever the routing."""
+    cfg = MoEConfig("t", T=16, H=64, I=32, E=6, k=3, bm=8, n_shared=1, bias=True, bias_mode="select",
+                    seed=19)
+    d = make_layer(cfg)
+    x, w13, w2 = to_numpy(d["x"]), to_numpy(d["w13"]), to_numpy(d["w2"])
+    w2[:cfg.E] = 0.0
+    out, _, _ = mo.moe_forward(x, to_numpy(d["logits"]), cfg.k, w13, w2, bias=to_numpy(d["bias"]),
+                               n_shared=1, bias_mode="select")
+    np.testing.assert_allclose(out, _dense_swiglu_bf16(x, w13[cfg.E], w2[cfg.E]), rtol=1e-5, atol=1e-6)
 
 
 @pytest.mark.parametrize("a8w8", [False, True])

@@ -3,7 +3,9 @@
 Gate: brute force over all k-subsets (the selected set is the one whose every
 member beats every non-member, ties to the lower index); the weights equal a
 library softmax over the selected logits alone; with k = E they are the full
-softmax; a bias is the same as shifting the logits.
+softmax; a bias is the same as shifting the logits; the selection-only bias
+picks by logit + bias and weighs by the raw logits (brute force, a constant
+bias, a bias that forces a set of experts).
 
 Align&sort: brute force with Python's ``sorted`` on (expert, slot) pairs and
 an explicit segment build; the structural invariants (non-sentinel entries
@@ -61,6 +63,64 @@ def test_gate_weights_sum_to_one_and_bias_shift():
     ids2, w2 = mo.topk_gate((logits + bias[None]).astype(np.float32), 8)
     np.testing.assert_array_equal(ids, ids2)
     np.testing.assert_array_equal(w, w2)
+
+
+@pytest.mark.parametrize("E,k", [(6, 2), (8, 3), (8, 8)])
+def test_gate_bias_modes_brute_force(E, k):
+    """Both bias modes select by brute force on logit + bias; "logits" weighs
+    the chosen experts by a softmax of logit + bias, "select" by a softmax of
+    the raw logits (library softmax over the chosen entries only)."""
+    rng = np.random.default_rng(100 + E * 10 + k)
+    logits = rng.integers(-3, 4, size=(150, E)).astype(np.float32)
+    bias = rng.integers(-2, 3, size=E).astype(np.float32)
+    score = logits + bias[None]
+    for mode in ("logits", "select"):
+        ids, w = mo.topk_gate(logits, k, bias, mode)
+        for t in range(logits.shape[0]):
+            assert list(ids[t]) == _brute_topk(list(score[t]), k)
+            src = score[t] if mode == "logits" else logits[t]
+            ref = scipy.special.softmax(src[ids[t]].astype(np.float64))
+            np.testing.assert_allclose(w[t], ref, rtol=1e-6, atol=1e-7)
+
+
+def test_gate_select_bias_constant_and_zero():
+    """A bias equal for every expert changes nothing in "select" mode (and in
+    "logits" mode the shift cancels in the softmax); a zero bias is no bias."""
+    rng = np.random.default_rng(5)
+    logits = rng.standard_normal((200, 64)).astype(np.float32)
+    ids0, w0 = mo.topk_gate(logits, 6)
+    for mode in ("select", "logits"):
+        ids, w = mo.topk_gate(logits, 6, np.zeros(64, np.float32), mode)
+        np.testing.assert_array_equal(ids, ids0)
+        np.testing.assert_array_equal(w, w0)
+    ids, w = mo.topk_gate(logits, 6, np.full(64, 0.5, np.float32), "select")
+    np.testing.assert_array_equal(ids, ids0)
+    np.testing.assert_allclose(w, w0, rtol=1e-6)
+
+
+def test_gate_select_bias_steers_only_selection():
+    """A large bias on a fixed set of k experts makes exactly that set the
+    choice (ordered by logit + bias) while the weights stay the softmax of the
+    raw logits of those experts."""
+    rng = np.random.default_rng(6)
+    E, k = 32, 4
+    logits = rng.standard_normal((100, E)).astype(np.float32)
+    favour = np.array([3, 11, 17, 29])
+    bias = np.zeros(E, np.float32)
+    bias[favour] = 1000.0 + np.arange(4, dtype=np.float32)
+    ids, w = mo.topk_gate(logits, k, bias, "select")
+    for t in range(100):
+        assert sorted(ids[t]) == sorted(favour)
+        ref = scipy.special.softmax(logits[t, ids[t]].astype(np.float64))
+        np.testing.assert_allclose(w[t], ref, rtol=1e-6, atol=1e-7)
+
+
+def test_add_shared_layout():
+    ids = np.array([[3, 1], [0, 2]], np.int32)
+    w = np.array([[0.7, 0.3], [0.6, 0.4]], np.float32)
+    ids2, w2 = mo.add_shared(ids, w, 4, 2)
+    np.testing.assert_array_equal(ids2, [[3, 1, 4, 5], [0, 2, 4, 5]])
+    np.testing.assert_array_equal(w2, np.array([[0.7, 0.3, 1, 1], [0.6, 0.4, 1, 1]], np.float32))
 
 
 def _brute_align(ids_flat, E, bm):
