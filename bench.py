@@ -54,8 +54,17 @@ def peaks():
 
 
 def workload_name(cfg, dtype):
+    bias = ""
+    if cfg.bias:
+        bias = " +bias(selection only)" if cfg.bias_mode == "select" else " +bias"
+    shared = f" +{cfg.n_shared} shared" if cfg.n_shared else ""
     return (f"{cfg.name}_{dtype}: T={cfg.T} H={cfg.H} I={cfg.I} E={cfg.E} k={cfg.k} bm={cfg.bm}"
-            f"{' +bias' if cfg.bias else ''}")
+            f"{bias}{shared}")
+
+
+def slot_pairs(cfg):
+    """(token, expert) pairs the FFN computes: k routed + the shared experts."""
+    return cfg.T * (cfg.k + cfg.n_shared)
 
 
 # ---------------------------------------------------------------------------
@@ -123,14 +132,15 @@ def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0):
     d = make_layer(cfg, device=dev)
     if cfg.a8w8:
         layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype,
-                           tile_tokens=tile_tokens)
+                           tile_tokens=tile_tokens, n_shared=cfg.n_shared, bias_mode=cfg.bias_mode)
     else:
-        layer = m.MoELayer(d["w13"], d["w2"], cfg.k, cfg.bm, out_dtype=out_dtype, tile_tokens=tile_tokens)
+        layer = m.MoELayer(d["w13"], d["w2"], cfg.k, cfg.bm, out_dtype=out_dtype, tile_tokens=tile_tokens,
+                           n_shared=cfg.n_shared, bias_mode=cfg.bias_mode)
     return d, layer
 
 
 def touched_experts(layer, d):
-    ids = torch.empty(d["x"].shape[0], layer.k, dtype=torch.int32, device=d["x"].device)
+    ids = torch.empty(d["x"].shape[0], layer.k + layer.n_shared, dtype=torch.int32, device=d["x"].device)
     layer(d["x"], d["logits"], d["bias"], topk_ids=ids)
     torch.cuda.synchronize()
     return int(torch.unique(ids).numel()), ids
@@ -145,7 +155,7 @@ def kernels_per_step(cfg, out_dtype):
     kernel of this library.)"""
     n = 5
     if cfg.a8w8:
-        n += 1 + (1 if cfg.T * cfg.k > 4096 else 0)
+        n += 1 + (1 if slot_pairs(cfg) > 4096 else 0)
     return n
 
 
@@ -224,14 +234,14 @@ def time_e2e(cfg, layer, d, steps, warmup):
 
 def gateup_bytes(cfg, touched):
     eb = 1 if cfg.a8w8 else 2
-    pairs = cfg.T * cfg.k
+    pairs = slot_pairs(cfg)
     w = touched * (2 * cfg.I * cfg.H * eb + (8 * cfg.I if cfg.a8w8 else 0))
     return w + pairs * cfg.H * eb + pairs * cfg.I * 2
 
 
 def down_bytes(cfg, touched):
     eb = 1 if cfg.a8w8 else 2
-    pairs = cfg.T * cfg.k
+    pairs = slot_pairs(cfg)
     w = touched * (cfg.H * cfg.I * eb + (4 * cfg.H if cfg.a8w8 else 0))
     return w + pairs * cfg.I * eb + pairs * cfg.H * 4     # + y, one fp32 row per slot
 
@@ -261,9 +271,9 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile
     ms_graph = time_graph(m, cfg, layer, d, steps, warmup)
     ms = ms_graph if ms_graph is not None else ms_eager
     step_ms = ms / steps
-    pairs = cfg.T * cfg.k
+    pairs = slot_pairs(cfg)
     fl = moe_flops(pairs, cfg.H, cfg.I)
-    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k, touched, cfg.I, cfg.a8w8)
+    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k + cfg.n_shared, touched, cfg.I, cfg.a8w8)
     tf_peak = pk["bf16_tflops_sustained"] * (2.0 if cfg.a8w8 else 1.0)
     t_roof = max(fl / (tf_peak * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
     rep = {"workload": workload_name(cfg, dtype_name), "tokens_per_s": cfg.T / (step_ms * 1e-3),
@@ -399,9 +409,9 @@ def run_ours(args):
     used_graph = graph is not None
     del graph
     step_ms = ms / args.steps
-    pairs = cfg.T * cfg.k
+    pairs = slot_pairs(cfg)
     fl = moe_flops(pairs, cfg.H, cfg.I)
-    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k, touched, cfg.I, False)
+    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k + cfg.n_shared, touched, cfg.I, False)
     t_roof = max(fl / (pk["bf16_tflops_sustained"] * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
     dom = max(stages, key=stages.get)
     kbytes = {"gateup": gateup_bytes(cfg, touched), "down": down_bytes(cfg, touched)}.get(dom)
@@ -423,6 +433,7 @@ def run_ours(args):
     if rank == 0 and not args.quick:
         extra["a8w8"], _, _ = layer_report(m, cfg.with_(a8w8=True), 50, 5, dev, pk, "a8w8")
         extra["mixtral"], _, _ = layer_report(m, CONFIGS["mixtral"], 20, 3, dev, pk, "bf16")
+        extra["deepseek_shared"], _, _ = layer_report(m, CONFIGS["deepseek_shared"], 50, 5, dev, pk, "bf16")
         extra["decode_a8w8"] = []
         for T in (1, 16, 64, 256):
             r, _, _ = layer_report(m, CONFIGS["decode"].with_(T=T), 100, 5, dev, pk, "a8w8")
@@ -555,6 +566,8 @@ def run_only(args):
     if parts[0] == "align":
         print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
         return
+    if len(parts) > 2 and f"{parts[0]}_{parts[1]}" in CONFIGS:     # e.g. deepseek_shared
+        parts = [f"{parts[0]}_{parts[1]}"] + parts[2:]
     cfg = CONFIGS[parts[0]].with_(a8w8=parts[1] == "a8w8")
     tile = 0
     for p in parts[2:]:
@@ -582,7 +595,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--only", default=None,
                     help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>][_E<N>][_tn<N>] "
-                         "(configs: tiny, p5, deepseek, mixtral, decode) or align_<T>")
+                         "(configs: tiny, p5, deepseek, deepseek_shared, mixtral, decode) or align_<T>")
     args = ap.parse_args()
     if args.only:
         run_only(args)

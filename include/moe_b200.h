@@ -79,19 +79,29 @@ MOE_API int moe_version(void);
  * moe_topk_gate -- softmax top-k gating.
  * Passage: MoE Align & Sort article, "FasterTransformer" (moe_softmax +
  * moe_top_k fused as topk_gating_softmax; "biased" variant) and the opening
- * definition (Top-K gating scores, a gating bias in DeepSeek V3).
+ * definition (Top-K gating scores; DeepSeek V3's gating bias for
+ * auxiliary-loss-free balancing and its shared expert).
  *
- *   logits   f32 [T, E]   router logits (the router GEMM is the caller's)
- *   bias     f32 [E]      nullable; added to the logits in fp32 before both
- *                         the selection and the softmax
- *   topk_ids i32 [T, k]   out: chosen experts, by descending (biased) logit;
- *                         equal logits go to the lower expert index
- *   topk_w   f32 [T, k]   out: softmax(l)[chosen] / sum(softmax(l)[chosen])
- * Limits: 0 <= T, 1 <= E <= 1024, 1 <= k <= min(E, 32).  Logits must be
- * finite.  Errors: MOE_ERR_INVALID_ARG on a bad size or NULL output.
+ *   logits    f32 [T, E]  router logits (the router GEMM is the caller's)
+ *   bias      f32 [E]     nullable; added to the logits in fp32
+ *   bias_mode             MOE_BIAS_LOGITS: the biased logits are both the
+ *                         selection score and the softmax input;
+ *                         MOE_BIAS_SELECT: they only select, the weights use
+ *                         the raw logits (DeepSeek-V3 style)
+ *   n_shared              shared experts appended to every token's row
+ *   topk_ids  i32 [T, k+n_shared]  out: chosen experts by descending score
+ *                         (equal scores go to the lower expert index), then
+ *                         the shared experts E, E+1, ..., E+n_shared-1
+ *   topk_w    f32 [T, k+n_shared]  out: softmax(l)[chosen] /
+ *                         sum(softmax(l)[chosen]), then 1 per shared expert
+ * Limits: 0 <= T, 1 <= E, E + n_shared <= 1024, 1 <= k <= E,
+ * k + n_shared <= 32, n_shared >= 0.  Logits must be finite.  Errors:
+ * MOE_ERR_INVALID_ARG on a bad size, mode or NULL output.
  * ------------------------------------------------------------------------- */
-MOE_API moe_status_t moe_topk_gate(const float* logits, const float* bias, int T, int E, int k,
-                           int32_t* topk_ids, float* topk_w, void* stream);
+#define MOE_BIAS_LOGITS 0
+#define MOE_BIAS_SELECT 1
+MOE_API moe_status_t moe_topk_gate(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
+                                   int n_shared, int32_t* topk_ids, float* topk_w, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_align_sort -- block-aligned MoE Align & Sort.
@@ -204,6 +214,12 @@ MOE_API moe_status_t moe_combine(const float* y, const float* topk_w, int T, int
  * the same arithmetic as moe_topk_gate, moe_align_sort, moe_grouped_ffn and
  * moe_combine in sequence (per-slot expert outputs kept in the workspace,
  * combined in fp32 in ascending j, so the result is deterministic).
+ * Shared experts (n_shared > 0; MoE Align & Sort article, opening: DeepSeek's
+ * shared expert) are stored after the E routed experts in w13/w2 and their
+ * scales ([E + n_shared, ...]); every token goes to each of them with weight
+ * 1, so they are scheduled in the same grouped GEMM launches as the routed
+ * experts (align & sort sees k + n_shared slots per token over
+ * E + n_shared experts).
  * ------------------------------------------------------------------------- */
 typedef struct {
   int T, H, I, E, k, block_size;
@@ -211,19 +227,22 @@ typedef struct {
   int out_dtype;              /* MOE_BF16 or MOE_F32                      */
   const void* x;              /* bf16 [T, H]                              */
   const float* logits;        /* f32 [T, E]                               */
-  const float* bias;          /* f32 [E], nullable                        */
-  const void* w13;            /* as in moe_ffn_args                       */
+  const float* bias;          /* f32 [E], nullable (see bias_mode)        */
+  const void* w13;            /* as in moe_ffn_args, E + n_shared experts */
   const float* w13_scale;
   const void* w2;
   const float* w2_scale;
   void* out;                  /* [T, H] out_dtype                         */
-  int32_t* topk_ids;          /* nullable: routing also written here [T,k] */
-  float* topk_w;              /* nullable [T,k]                           */
+  int32_t* topk_ids;          /* nullable: routing also written here
+                                 [T, k + n_shared] (as moe_topk_gate)      */
+  float* topk_w;              /* nullable [T, k + n_shared]               */
   int tile_tokens;            /* as in moe_ffn_args                       */
   void** stage_events;        /* nullable: MOE_NUM_STAGES + 1 cudaEvent_t
                                  handles; event 0 is recorded before the first
                                  stage and event i+1 after stage i, on
                                  `stream` (for per-stage timing)           */
+  int n_shared;               /* shared experts after the E routed ones (0..) */
+  int bias_mode;              /* MOE_BIAS_LOGITS or MOE_BIAS_SELECT        */
 } moe_forward_args;
 
 /* Stages of moe_forward, in launch order (stage_events indices). */

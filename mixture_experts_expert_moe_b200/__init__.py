@@ -42,7 +42,12 @@ class ForwardArgs(ctypes.Structure):
     _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i),
                 ("wdtype", _i), ("out_dtype", _i), ("x", _vp), ("logits", _vp), ("bias", _vp),
                 ("w13", _vp), ("w13_scale", _vp), ("w2", _vp), ("w2_scale", _vp), ("out", _vp),
-                ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i), ("stage_events", _vp)]
+                ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i), ("stage_events", _vp),
+                ("n_shared", _i), ("bias_mode", _i)]
+
+
+MOE_BIAS_LOGITS, MOE_BIAS_SELECT = 0, 1
+_BIAS_MODES = {"logits": MOE_BIAS_LOGITS, "select": MOE_BIAS_SELECT}
 
 
 _LIB = None
@@ -61,7 +66,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_status_string": (ctypes.c_char_p, [_i]),
             "moe_last_cuda_error": (ctypes.c_char_p, []),
             "moe_version": (_i, []),
-            "moe_topk_gate": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+            "moe_topk_gate": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
             "moe_align_sort_sizes": (_i, [_i, _i, _i, _i, sz, sz, sz]),
             "moe_align_sort": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]),
             "moe_ffn_workspace": (_i, [ctypes.POINTER(FfnArgs), sz]),
@@ -120,15 +125,19 @@ def _wdtype(w):
 # ops
 # ---------------------------------------------------------------------------
 
-def topk_gate(logits: torch.Tensor, k: int, bias: torch.Tensor | None = None):
-    """Softmax top-k gating: returns (ids int32 [T,k], weights f32 [T,k])."""
+def topk_gate(logits: torch.Tensor, k: int, bias: torch.Tensor | None = None, bias_mode: str = "logits",
+              n_shared: int = 0):
+    """Softmax top-k gating: returns (ids int32 [T, k+n_shared], weights f32
+    [T, k+n_shared]); the last n_shared columns are the shared experts E..
+    with weight 1.  bias_mode "logits": the bias shifts the logits for both
+    the choice and the weights; "select": it only steers the choice."""
     lib = load_library()
     assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous()
     T, E = logits.shape
-    ids = torch.empty(T, k, dtype=torch.int32, device=logits.device)
-    w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
-    _check(lib.moe_topk_gate(_ptr(logits), _ptr(bias), T, E, k, _ptr(ids), _ptr(w),
-                             _stream(logits.device)), "moe_topk_gate")
+    ids = torch.empty(T, k + n_shared, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, k + n_shared, dtype=torch.float32, device=logits.device)
+    _check(lib.moe_topk_gate(_ptr(logits), _ptr(bias), _BIAS_MODES[bias_mode], T, E, k, n_shared, _ptr(ids),
+                             _ptr(w), _stream(logits.device)), "moe_topk_gate")
     return ids, w
 
 
@@ -207,17 +216,22 @@ def combine(y: torch.Tensor, topk_w: torch.Tensor, out_dtype=torch.bfloat16, out
 class MoELayer:
     """One MoE layer forward through ``moe_forward`` with a reusable workspace.
 
-    Weights: ``w13 [E, 2I, H]`` (gate rows then up rows) and ``w2 [E, H, I]``,
-    bf16, or float8_e4m3fn codes with f32 per-row scales ``w13_scale [E, 2I]``
-    and ``w2_scale [E, H]``.
+    Weights: ``w13 [E + n_shared, 2I, H]`` (gate rows then up rows) and
+    ``w2 [E + n_shared, H, I]``, bf16, or float8_e4m3fn codes with f32 per-row
+    scales ``w13_scale [E + n_shared, 2I]`` and ``w2_scale [E + n_shared, H]``;
+    the last ``n_shared`` experts are shared (every token, weight 1).
+    ``bias_mode``: "logits" (the bias shifts the logits for the choice and the
+    weights) or "select" (it only steers the choice).
     """
 
     def __init__(self, w13, w2, k, block_size, w13_scale=None, w2_scale=None, out_dtype=torch.bfloat16,
-                 tile_tokens=0):
+                 tile_tokens=0, n_shared=0, bias_mode="logits"):
         self.w13, self.w2, self.k, self.block_size = w13, w2, k, block_size
         self.w13_scale, self.w2_scale = w13_scale, w2_scale
         self.out_dtype, self.tile_tokens = out_dtype, tile_tokens
-        self.E, twoI, self.H = w13.shape
+        self.n_shared, self.bias_mode = n_shared, _BIAS_MODES[bias_mode]
+        EW, twoI, self.H = w13.shape
+        self.E = EW - n_shared
         self.I = twoI // 2
         self._ws = None
 
@@ -231,14 +245,15 @@ class MoELayer:
             w2=self.w2.data_ptr(), w2_scale=None if self.w2_scale is None else self.w2_scale.data_ptr(),
             out=out.data_ptr(), topk_ids=None if ids is None else ids.data_ptr(),
             topk_w=None if w is None else w.data_ptr(), tile_tokens=self.tile_tokens,
-            stage_events=None if events is None else ctypes.cast(events, ctypes.c_void_p))
+            stage_events=None if events is None else ctypes.cast(events, ctypes.c_void_p),
+            n_shared=self.n_shared, bias_mode=self.bias_mode)
 
     def workspace_bytes(self, T):
         lib = load_library()
         a = ForwardArgs(T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
                         wdtype=_wdtype(self.w13),
                         out_dtype=MOE_BF16 if self.out_dtype == torch.bfloat16 else MOE_F32,
-                        tile_tokens=self.tile_tokens)
+                        tile_tokens=self.tile_tokens, n_shared=self.n_shared, bias_mode=self.bias_mode)
         n = ctypes.c_size_t()
         _check(lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)), "moe_forward_workspace")
         return n.value

@@ -149,7 +149,8 @@ __device__ __forceinline__ bool validate_keys(long long base, long long end, int
 
 // EPL = ceil(E/32) rounded up to a power of two (the gating's logits per lane
 // and the width of the id matching).  kGate: the CTA first gates the tokens
-// whose slots it owns (its chunk is a multiple of k) and writes ids/weights.  kPlan: CTA 0 finally writes the
+// whose slots it owns (its chunk is a multiple of the slots per token) and
+// writes ids/weights.  kPlan: CTA 0 finally writes the
 // grouped GEMMs' tile plan from the padded offsets.  With one CTA there is no
 // grid-wide wait.
 template <int EPL, bool kGate, bool kPlan>
@@ -170,10 +171,12 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   const long long cta_begin = (long long)blockIdx.x * p.chunk;
   if (kGate) {
     // ---- gating of this CTA's tokens (warp per token) ----------------------
-    const long long t0 = cta_begin / r.k;
-    const long long t1 = min((long long)r.T, (cta_begin + p.chunk) / r.k);
+    const int kk = r.k + r.n_shared;   // slots per token
+    const long long t0 = cta_begin / kk;
+    const long long t1 = min((long long)r.T, (cta_begin + p.chunk) / kk);
     for (long long t = t0 + warp; t < t1; t += kAlignWarps)
-      gate_token<EPL>(r.logits, r.bias, t, E, r.k, r.ids_out, r.w_out, lane);
+      gate_token<EPL>(r.logits, r.bias, r.select_only != 0, t, r.E_routed, r.k, r.n_shared, r.ids_out, r.w_out,
+                      lane);
   }
   __syncthreads();
 

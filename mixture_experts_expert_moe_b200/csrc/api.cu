@@ -253,9 +253,11 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
 }
 
 // Gate + align&sort + tile plan in one launch (moe_forward).
-moe_status_t run_route(const FfnShape& s, const float* logits, const float* bias, int32_t* ids, float* w,
-                       int32_t* sorted, int32_t* expert_ids, int32_t* num_post, void* align_ws, int32_t* plan,
-                       int32_t* status, cudaStream_t stream) {
+// s holds the expert and slot counts with the shared experts included
+// (s.E = E_routed + n_shared, s.k = k_routed + n_shared).
+moe_status_t run_route(const FfnShape& s, int n_shared, bool select_only, const float* logits, const float* bias,
+                       int32_t* ids, float* w, int32_t* sorted, int32_t* expert_ids, int32_t* num_post,
+                       void* align_ws, int32_t* plan, int32_t* status, cudaStream_t stream) {
   const int N = (int)s.N;
   int err = 0;
   const int max_ctas = moe::align_max_ctas(s.E, &err);
@@ -296,8 +298,11 @@ moe_status_t run_route(const FfnShape& s, const float* logits, const float* bias
   moe::RouteExtra r;
   r.logits = logits;
   r.bias = bias;
+  r.select_only = select_only ? 1 : 0;
   r.T = s.T;
-  r.k = s.k;
+  r.k = s.k - n_shared;
+  r.E_routed = s.E - n_shared;
+  r.n_shared = n_shared;
   r.ids_out = ids;
   r.w_out = w;
   r.plan = plan;
@@ -329,14 +334,17 @@ const char* moe_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
 int moe_version(void) { return 100; }
 
-moe_status_t moe_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* topk_ids,
-                           float* topk_w, void* stream) {
-  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+moe_status_t moe_topk_gate(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
+                           int n_shared, int32_t* topk_ids, float* topk_w, void* stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || n_shared < 0 || k + n_shared > 32 || E + n_shared > 1024)
+    return MOE_ERR_INVALID_ARG;
+  if (bias_mode != MOE_BIAS_LOGITS && bias_mode != MOE_BIAS_SELECT) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   moe_status_t st = check_device();
   if (st) return st;
-  MOE_CU(moe::launch_topk_gate(logits, bias, T, E, k, topk_ids, topk_w, (cudaStream_t)stream));
+  MOE_CU(moe::launch_topk_gate(logits, bias, bias_mode == MOE_BIAS_SELECT, T, E, k, n_shared, topk_ids, topk_w,
+                               (cudaStream_t)stream));
   return MOE_OK;
 }
 
@@ -422,11 +430,21 @@ FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
 }
 }  // namespace
 
+// Shape of a forward call: the shared experts count as experts and as slots.
+moe_status_t forward_shape(const moe_forward_args* a, FfnShape* s) {
+  if (a->out_dtype != MOE_BF16 && a->out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (a->bias_mode != MOE_BIAS_LOGITS && a->bias_mode != MOE_BIAS_SELECT) return MOE_ERR_INVALID_ARG;
+  if (a->n_shared < 0 || a->E < 1 || a->k < 1 || a->k > a->E || a->k + a->n_shared > 32 ||
+      a->E + a->n_shared > 1024)
+    return MOE_ERR_INVALID_ARG;
+  return ffn_shape(a->T, a->H, a->I, a->E + a->n_shared, a->k + a->n_shared, a->block_size, a->wdtype,
+                   a->tile_tokens, s);
+}
+
 moe_status_t moe_forward_workspace(const moe_forward_args* a, size_t* ws_bytes) {
   if (!a || !ws_bytes) return MOE_ERR_INVALID_ARG;
-  if (a->out_dtype != MOE_BF16 && a->out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   FfnShape s;
-  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  moe_status_t st = forward_shape(a, &s);
   if (st) return st;
   *ws_bytes = fwd_ws_layout(s, a->out_dtype).total;
   return MOE_OK;
@@ -435,9 +453,8 @@ moe_status_t moe_forward_workspace(const moe_forward_args* a, size_t* ws_bytes) 
 moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
                          void* stream) {
   if (!a) return MOE_ERR_INVALID_ARG;
-  if (a->out_dtype != MOE_BF16 && a->out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   FfnShape s;
-  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
+  moe_status_t st = forward_shape(a, &s);
   if (st) return st;
   if (s.T == 0) return MOE_OK;
   if (!a->x || !a->logits || !a->w13 || !a->w2 || !a->out || !ws) return MOE_ERR_INVALID_ARG;
@@ -461,7 +478,8 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   // gate, align&sort and the GEMM tile plan are one launch: stages 0..2 end together
   uint8_t* ffn_ws = w + L.ffn;
   int32_t* plan = reinterpret_cast<int32_t*>(ffn_ws + ffn_ws_layout(s).plan);
-  st = run_route(s, a->logits, a->bias, ids, tw, sorted, eids, npost, w + L.align, plan, dev_status, cs);
+  st = run_route(s, a->n_shared, a->bias_mode == MOE_BIAS_SELECT, a->logits, a->bias, ids, tw, sorted, eids, npost,
+                 w + L.align, plan, dev_status, cs);
   if (st) return st;
   MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));

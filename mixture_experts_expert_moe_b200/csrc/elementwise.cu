@@ -18,25 +18,28 @@ namespace moe {
 // ---------------------------------------------------------------------------
 template <int EPL>
 __global__ void __launch_bounds__(256) topk_gate_kernel(const float* __restrict__ logits,
-                                                        const float* __restrict__ bias, int T, int E, int k,
-                                                        int32_t* __restrict__ ids, float* __restrict__ w) {
+                                                        const float* __restrict__ bias, bool select_only, int T,
+                                                        int E, int k, int n_shared, int32_t* __restrict__ ids,
+                                                        float* __restrict__ w) {
   const long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  gate_token<EPL>(logits, bias, t, E, k, ids, w, threadIdx.x & 31);
+  gate_token<EPL>(logits, bias, select_only, t, E, k, n_shared, ids, w, threadIdx.x & 31);
 }
 
-cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* ids,
-                             float* w, cudaStream_t s) {
+cudaError_t launch_topk_gate(const float* logits, const float* bias, bool select_only, int T, int E, int k,
+                             int n_shared, int32_t* ids, float* w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   dim3 grid((unsigned)((T + warps - 1) / warps)), block(32 * warps);
   const int epl = (E + 31) / 32;
-  if (epl <= 1) topk_gate_kernel<1><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
-  else if (epl <= 2) topk_gate_kernel<2><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
-  else if (epl <= 4) topk_gate_kernel<4><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
-  else if (epl <= 8) topk_gate_kernel<8><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
-  else if (epl <= 16) topk_gate_kernel<16><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
-  else topk_gate_kernel<32><<<grid, block, 0, s>>>(logits, bias, T, E, k, ids, w);
+#define MOE_GATE(V) topk_gate_kernel<V><<<grid, block, 0, s>>>(logits, bias, select_only, T, E, k, n_shared, ids, w)
+  if (epl <= 1) MOE_GATE(1);
+  else if (epl <= 2) MOE_GATE(2);
+  else if (epl <= 4) MOE_GATE(4);
+  else if (epl <= 8) MOE_GATE(8);
+  else if (epl <= 16) MOE_GATE(16);
+  else MOE_GATE(32);
+#undef MOE_GATE
   return cudaGetLastError();
 }
 

@@ -22,24 +22,28 @@ struct AlignParams {
 
 // Extra inputs of the fused routing launch (gating in front, tile plan behind).
 struct RouteExtra {
-  const float* logits;  // [T, E]
-  const float* bias;    // [E] or null
-  int T, k;
-  int32_t* ids_out;     // [T*k] (the same buffer AlignParams::ids reads)
-  float* w_out;         // [T*k]
+  const float* logits;  // [T, E_routed]
+  const float* bias;    // [E_routed] or null
+  int select_only;      // the bias steers the selection only
+  int T, k;             // tokens, routed choices per token
+  int E_routed;         // routed experts; AlignParams::E = E_routed + n_shared
+  int n_shared;         // shared experts (every token, weight 1)
+  int32_t* ids_out;     // [T*(k+n_shared)] (the same buffer AlignParams::ids reads)
+  float* w_out;         // [T*(k+n_shared)]
   int32_t* plan;        // plan layout below
   int tn, nw_gu, nw_dn;
 };
 
 size_t align_smem_bytes(int E);
 cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream);
-// gate + align&sort + tile plan in one cooperative launch (p.chunk % k == 0)
+// gate + align&sort + tile plan in one cooperative launch (p.chunk % (k + n_shared) == 0)
 cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream);
 int align_max_ctas(int E, int* err_out);
 cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout_ns, cudaStream_t stream);
 
-cudaError_t launch_topk_gate(const float* logits, const float* bias, int T, int E, int k, int32_t* ids,
-                             float* w, cudaStream_t s);
+// ids/w rows of k + n_shared entries (the shared experts E.. with weight 1)
+cudaError_t launch_topk_gate(const float* logits, const float* bias, bool select_only, int T, int E, int k,
+                             int n_shared, int32_t* ids, float* w, cudaStream_t s);
 // dst row r = src row sorted[r]/k (row_bytes each, a multiple of 16), zero for
 // padding; with scales also dst_scale[r] = src_scale[token] (1 for padding)
 cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,

@@ -46,12 +46,34 @@ def test_align_sizes():
     assert lib.moe_align_sort_sizes(-1, 2, 8, 16, ctypes.byref(P), None, None) == 1
 
 
-@pytest.mark.parametrize("bad", [dict(E=0), dict(k=0), dict(k=9), dict(T=-1), dict(E=1025)])
+@pytest.mark.parametrize("bad", [dict(E=0), dict(k=0), dict(k=9), dict(T=-1), dict(E=1025), dict(mode=2),
+                                 dict(mode=-1), dict(S=-1), dict(k=8, E=40, S=25), dict(E=1020, S=5)])
 def test_gate_rejects_bad_sizes(bad):
     lib = m.load_library()
-    a = dict(T=4, E=8, k=2)
+    a = dict(T=4, E=8, k=2, mode=0, S=0)
     a.update(bad)
-    assert lib.moe_topk_gate(None, None, a["T"], a["E"], a["k"], None, None, None) == 1
+    assert lib.moe_topk_gate(None, None, a["mode"], a["T"], a["E"], a["k"], a["S"], None, None, None) == 1
+
+
+@pytest.mark.parametrize("bad", [dict(bias_mode=2), dict(n_shared=-1), dict(n_shared=31), dict(E=1024, n_shared=1)])
+def test_forward_workspace_rejects_bad_shared_and_mode(bad):
+    lib = m.load_library()
+    a = dict(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, out_dtype=0, tile_tokens=0, n_shared=0,
+             bias_mode=0)
+    a.update(bad)
+    n = ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(m.ForwardArgs(**a)), ctypes.byref(n)) == 1
+
+
+def test_forward_workspace_counts_shared_slots():
+    """A shared expert adds one slot per token and one expert: the workspace
+    grows accordingly."""
+    lib = m.load_library()
+    base = dict(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, out_dtype=0, tile_tokens=0)
+    n0, n1 = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(m.ForwardArgs(**base)), ctypes.byref(n0)) == 0
+    assert lib.moe_forward_workspace(ctypes.byref(m.ForwardArgs(**base, n_shared=1)), ctypes.byref(n1)) == 0
+    assert n1.value > n0.value
 
 
 def _ffn(**kw):

@@ -106,6 +106,44 @@ def test_forward_parity_small(cuda_device, cfg, a8w8):
         assert_close(out.float().cpu().numpy(), ref, tol, f"{cfg.name} out {out_dtype}")
 
 
+SHARED = [
+    # DeepSeek-style: selection-only bias and one shared expert
+    MoEConfig("shared1", T=300, H=384, I=256, E=16, k=4, bm=32, bias=True, n_shared=1, bias_mode="select",
+              seed=106),
+    MoEConfig("shared2", T=64, H=256, I=128, E=8, k=2, bm=16, bias=True, n_shared=2, seed=107),
+    # shared expert with many tokens next to routed experts with few
+    MoEConfig("shared_big", T=700, H=512, I=384, E=32, k=2, bm=64, n_shared=1, bias=True, bias_mode="select",
+              seed=108),
+]
+
+
+@pytest.mark.parametrize("a8w8", [False, True])
+@pytest.mark.parametrize("cfg", SHARED, ids=lambda c: c.name)
+def test_forward_parity_shared_and_bias_modes(cuda_device, cfg, a8w8):
+    cfg = cfg.with_(a8w8=a8w8)
+    d = make_layer(cfg)
+    g = _dev(d, cuda_device)
+    w13, w2, s13, s2 = _weights(cfg, g)
+    ref, ref_ids, ref_w = oracle.moe_forward(
+        to_numpy(d["x"]), to_numpy(d["logits"]), cfg.k,
+        to_numpy(d["w13_q"] if a8w8 else d["w13"]), to_numpy(d["w2_q"] if a8w8 else d["w2"]),
+        bias=to_numpy(d["bias"]), a8w8=a8w8, w13_s=to_numpy(d.get("w13_s")), w2_s=to_numpy(d.get("w2_s")),
+        n_shared=cfg.n_shared, bias_mode=cfg.bias_mode)
+    tol = TOL_FP8 if a8w8 else TOL_BF16
+    kk = cfg.k + cfg.n_shared
+    layer = m.MoELayer(w13, w2, cfg.k, cfg.bm, s13, s2, out_dtype=torch.float32, n_shared=cfg.n_shared,
+                       bias_mode=cfg.bias_mode)
+    ids = torch.empty(cfg.T, kk, dtype=torch.int32, device=cuda_device)
+    tw = torch.empty(cfg.T, kk, dtype=torch.float32, device=cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = layer(g["x"], g["logits"], g["bias"], topk_ids=ids, topk_w=tw, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.max(np.abs(tw.cpu().numpy() - ref_w)) <= 1e-6
+    assert_close(out.float().cpu().numpy(), ref, tol, f"{cfg.name} out")
+
+
 def test_forward_zero_input(cuda_device):
     cfg = SMALL[1]
     d = make_layer(cfg)

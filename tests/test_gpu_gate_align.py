@@ -43,6 +43,20 @@ def test_topk_gate_parity(cuda_device, T, E, k, bias, ties):
         assert np.max(np.abs(w.cpu().numpy().astype(np.float64) - ref_w)) <= 1e-6
 
 
+@pytest.mark.parametrize("T,E,k,n_shared,mode", [
+    (2048, 256, 8, 1, "select"), (2048, 256, 8, 0, "select"), (300, 33, 5, 2, "select"),
+    (300, 33, 5, 2, "logits"), (64, 8, 2, 3, "logits"), (777, 64, 8, 1, "select"), (40, 1000, 24, 8, "select"),
+])
+def test_topk_gate_bias_modes_and_shared(cuda_device, T, E, k, n_shared, mode):
+    logits, b = _gate_case(T, E, k, True, seed=T * 11 + E + n_shared, ties=False)
+    ids, w = m.topk_gate(logits.to(cuda_device), k, b.to(cuda_device), bias_mode=mode, n_shared=n_shared)
+    torch.cuda.synchronize()
+    ref_ids, ref_w = oracle.topk_gate(logits.numpy(), k, b.numpy(), mode)
+    ref_ids, ref_w = oracle.add_shared(ref_ids, ref_w, E, n_shared)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.max(np.abs(w.cpu().numpy().astype(np.float64) - ref_w)) <= 1e-6
+
+
 def _align_case(T, k, E, bm, dist, seed):
     if dist == "same":
         return np.zeros((T, k), np.int32) + (E - 1)
