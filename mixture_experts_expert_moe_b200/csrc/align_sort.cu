@@ -347,6 +347,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
       r.plan[5 + 5 * E] = td;
       r.plan[0] = tg;
       r.plan[1] = td;
+      r.plan[plan_counter(E, true)] = 0;
+      r.plan[plan_counter(E, false)] = 0;
       r.plan[2] = r.tn;
       r.plan[3] = total_post;
     }

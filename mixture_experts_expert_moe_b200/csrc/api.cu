@@ -219,6 +219,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.out = h;
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g1.p.tile_counter = plan + moe::plan_counter(s.E, true);
   int r = moe::launch_grouped_gemm(g1, stream);
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
@@ -246,6 +247,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.out = y;
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g2.p.tile_counter = plan + moe::plan_counter(s.E, false);
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));

@@ -36,6 +36,7 @@ constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilog
 constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
+constexpr int kRing = 4;         // tile indices in flight from the producer to the other warps
 
 // Plan layout (int32), written by plan_kernel from the align&sort outputs.
 //   [0] tiles of the gate/up GEMM   [1] tiles of the down GEMM   [2] tn
@@ -44,6 +45,7 @@ constexpr int kWTileBytes = kWRows * kStageK;
 //   groups[E]    @4+2E   token groups of <= tn rows
 //   pref_gu[E+1] @4+3E   exclusive prefix of gate/up tiles per expert
 //   pref_dn[E+1] @5+4E   exclusive prefix of down tiles per expert
+//   counters     @6+5E   tiles claimed so far by the gate/up and the down GEMM
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ expert_ids,
                                                     const int32_t* __restrict__ num_post, int P, int E, int bm,
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     plan[1] = b;
     plan[2] = tn;
     plan[3] = np;
+    plan[plan_counter(E, true)] = 0;
+    plan[plan_counter(E, false)] = 0;
   }
 }
 
@@ -169,9 +173,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = bars + 2 * p.stages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* t_full = drain + 1;          // [kRing] a tile index was published
+  uint64_t* t_empty = t_full + kRing;    // [kRing] every consumer has read it
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(t_empty + kRing);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  int* s_start = s_abort + 3;   // keep 16-byte alignment of the arrays below
+  int* s_ring = s_abort + 1;    // [kRing]
+  int* s_start = s_ring + kRing + 2;
   int* s_rows = s_start + E;
   int* s_groups = s_rows + E;
   int* s_pref = s_groups + E;   // E + 1
@@ -188,6 +195,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&t_full[r], 1);
+      mbar_init(&t_empty[r], 9);   // the MMA thread and the 8 epilogue warps
+    }
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
@@ -225,7 +236,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       long long armed = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int it = 0; ok; ++it) {
+        // claim the next tile of the launch and publish it to the MMA and epilogue warps
+        const int slot = it % kRing;
+        if (!wait_or_abort(&t_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u, p.timeout_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int t = atomicAdd(p.tile_counter, 1);
+        s_ring[slot] = t;
+        mbar_arrive(&t_full[slot]);
+        if (t >= n_tiles) break;
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         int row0, row1;
         bool has1 = true;
@@ -281,7 +302,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       const uint32_t fmt = p.fp8 ? 0u : 1u;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+      for (;; ++it) {
+        const int slot = it % kRing;
+        if (!wait_or_abort(&t_full[slot], (uint32_t)(it / kRing) & 1u, p.timeout_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int t = s_ring[slot];
+        mbar_arrive(&t_empty[slot]);
+        if (t >= n_tiles) break;
         const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
         const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
@@ -340,8 +369,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int m = 32 * q + lane;
-    int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+    for (int it = 0;; ++it) {
+      const int slot = it % kRing;
+      if (!wait_or_abort(&t_full[slot], (uint32_t)(it / kRing) & 1u, p.timeout_ns, abort_flag)) break;
+      const int t = s_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[slot]);
+      if (t >= n_tiles) break;
       const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
       const int acc = it % p.n_acc;
       const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
@@ -463,7 +497,8 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, long long
 size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
   const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
   (void)gateup;
-  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 6) * 8 + 16 + (size_t)(4 * E + 1) * 4;
+  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5 + 2 * kRing) * 8 + (kRing + 4) * 4 +
+         (size_t)(4 * E + 1) * 4;
 }
 
 int gemm_pick_stages(int gateup, int tn, int E) {

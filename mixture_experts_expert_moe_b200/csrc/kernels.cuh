@@ -62,7 +62,10 @@ cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, 
 //   [0] gate/up tiles  [1] down tiles  [2] tokens per tile  [3] padded rows
 //   seg_start[E] @4, seg_rows[E] @4+E, groups[E] @4+2E,
 //   pref_gu[E+1] @4+3E, pref_dn[E+1] @5+4E
-__host__ __device__ inline int plan_ints(int E) { return 6 + 5 * E; }
+// + two tile counters ([6+5E] gate/up, [7+5E] down) that the plan writer zeroes
+// and the GEMM launches take tiles from
+__host__ __device__ inline int plan_ints(int E) { return 8 + 5 * E; }
+__host__ __device__ inline int plan_counter(int E, bool gateup) { return gateup ? 6 + 5 * E : 7 + 5 * E; }
 cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
                         int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s);
 
@@ -85,6 +88,7 @@ struct GemmParams {
   void* out;             // gate/up: h bf16 [P, n_out]; down: y f32 [T*k, n_out] (one row per slot)
   int32_t* status;
   long long timeout_ns;
+  int* tile_counter;     // next unclaimed tile of this launch (zero at launch)
 };
 
 struct GemmLaunch {
