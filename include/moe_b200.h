@@ -212,8 +212,12 @@ MOE_API moe_status_t moe_combine(const float* y, const float* topk_w, int T, int
 /* ---------------------------------------------------------------------------
  * moe_forward -- gate, align & sort, grouped FFN and combine in one call:
  * the same arithmetic as moe_topk_gate, moe_align_sort, moe_grouped_ffn and
- * moe_combine in sequence (per-slot expert outputs kept in the workspace,
- * combined in fp32 in ascending j, so the result is deterministic).
+ * moe_combine in sequence.  With k + n_shared >= 4 slots per token the
+ * combine is fused into the down GEMM: each slot's w * y is added into an
+ * fp32 row per token (in L2, in no fixed order, so the last bits of the
+ * output may differ between calls), then rounded once to out_dtype.  With
+ * fewer slots the per-slot outputs are summed by the combine kernel in
+ * ascending j (deterministic).
  * Shared experts (n_shared > 0; MoE Align & Sort article, opening: DeepSeek's
  * shared expert) are stored after the E routed experts in w13/w2 and their
  * scales ([E + n_shared, ...]); every token goes to each of them with weight
@@ -252,8 +256,9 @@ typedef struct {
 #define MOE_STAGE_GATHER 3    /* token rows to sorted order (+FP8 quant)   */
 #define MOE_STAGE_GATEUP 4    /* gate/up GEMM with SiLU*mul                */
 #define MOE_STAGE_REQUANT 5   /* FP8 requantisation of h (empty for bf16)  */
-#define MOE_STAGE_DOWN 6      /* down GEMM, one fp32 row per slot          */
-#define MOE_STAGE_COMBINE 7   /* top-k weighted combine into out           */
+#define MOE_STAGE_DOWN 6      /* down GEMM (with the combine when fused)    */
+#define MOE_STAGE_COMBINE 7   /* combine kernel, or the fp32 -> bf16 rounding
+                                 of the fused accumulator (empty for f32)    */
 #define MOE_NUM_STAGES 8
 
 MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);

@@ -171,7 +171,7 @@ moe_status_t gemm_fail(int r, const char* what) {
 moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
                      const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
                      float* y, uint8_t* ws, int32_t* status, cudaStream_t stream, void** ev = nullptr,
-                     bool plan_ready = false) {
+                     bool plan_ready = false, float* comb_out = nullptr, const float* comb_w = nullptr) {
   const FfnWs L = ffn_ws_layout(s);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
@@ -248,6 +248,8 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g2.p.status = status;
   g2.p.timeout_ns = moe::kDefaultTimeoutNs;
   g2.p.tile_counter = plan + moe::plan_counter(s.E, false);
+  g2.p.comb_out = comb_out;   // non-null: out32[t] += w * y in the epilogue, y is not written
+  g2.p.comb_w = comb_w;
   r = moe::launch_grouped_gemm(g2, stream);
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
@@ -412,8 +414,18 @@ moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int 
 }
 
 namespace {
+// The combine is fused into the down GEMM's epilogue when a token has at
+// least this many slots (then the per-slot outputs are >= 4x the token
+// outputs).  With fewer slots the per-slot round trip is small, and the down
+// GEMM's re-read operands (h, weights) need L2 more than an fp32 token
+// accumulator does (measured: Mixtral, k = 2, is faster unfused; DeepSeek-V3,
+// k = 8, fused).
+constexpr int kFuseCombineMinSlots = 4;
+
+bool fuse_combine(const FfnShape& s) { return s.k >= kFuseCombineMinSlots; }
+
 struct FwdWs {
-  size_t ids, w, sorted, eids, npost, align, ffn, y, total;
+  size_t ids, w, sorted, eids, npost, align, ffn, acc, y, total;
 };
 FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
   Carver c;
@@ -425,8 +437,11 @@ FwdWs fwd_ws_layout(const FfnShape& s, int out_dtype) {
   w.npost = c.take(4);
   w.align = c.take(align_ws_bytes(s.E));
   w.ffn = c.take(ffn_ws_layout(s).total);
-  w.y = c.take((size_t)s.N * s.H * 4);
-  (void)out_dtype;
+  // fused combine: fp32 token accumulator (the output itself when it is f32);
+  // otherwise one fp32 row per slot for the combine kernel
+  const bool fused = fuse_combine(s);
+  w.acc = c.take(fused && out_dtype == MOE_BF16 ? (size_t)s.T * s.H * 4 : 0);
+  w.y = c.take(fused ? 0 : (size_t)s.N * s.H * 4);
   w.total = c.off;
   return w;
 }
@@ -475,8 +490,12 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   int32_t* eids = reinterpret_cast<int32_t*>(w + L.eids);
   int32_t* npost = reinterpret_cast<int32_t*>(w + L.npost);
   void** ev = a->stage_events;
-  float* y = reinterpret_cast<float*>(w + L.y);
+  const bool out_bf16 = a->out_dtype == MOE_BF16;
+  const bool fused = fuse_combine(s);
+  float* out32 = !fused ? nullptr : out_bf16 ? reinterpret_cast<float*>(w + L.acc) : static_cast<float*>(a->out);
+  float* y = fused ? nullptr : reinterpret_cast<float*>(w + L.y);
   MOE_CU(record(ev, 0, cs));
+  if (fused) MOE_CU(cudaMemsetAsync(out32, 0, (size_t)s.T * s.H * 4, cs));
   // gate, align&sort and the GEMM tile plan are one launch: stages 0..2 end together
   uint8_t* ffn_ws = w + L.ffn;
   int32_t* plan = reinterpret_cast<int32_t*>(ffn_ws + ffn_ws_layout(s).plan);
@@ -485,10 +504,16 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   if (st) return st;
   MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
+  // fused: the down GEMM adds w * y of every slot into its token's fp32 row;
+  // otherwise it writes y per slot and the combine kernel sums them
   st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, y, ffn_ws, dev_status,
-               cs, ev, /*plan_ready=*/true);
+               cs, ev, /*plan_ready=*/true, out32, tw);
   if (st) return st;
-  MOE_CU(moe::launch_combine(y, tw, s.T, s.k, s.H, a->out, a->out_dtype == MOE_BF16, cs));
+  if (fused) {
+    if (out_bf16) MOE_CU(moe::launch_cast_bf16(out32, (long long)s.T * s.H, a->out, cs));
+  } else {
+    MOE_CU(moe::launch_combine(y, tw, s.T, s.k, s.H, a->out, out_bf16, cs));
+  }
   MOE_CU(record(ev, MOE_STAGE_COMBINE + 1, cs));
   return MOE_OK;
 }

@@ -400,6 +400,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   }
 }
 
+// fp32 -> bf16 (round to nearest even), n a multiple of 4, 16-byte aligned
+__global__ void __launch_bounds__(256) cast_bf16_kernel(const float4* __restrict__ src, long long n4,
+                                                        uint2* __restrict__ dst) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = __ldg(src + i);
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t*>(&a);
+    o.y = *reinterpret_cast<uint32_t*>(&b);
+    dst[i] = o;
+  }
+}
+
+cudaError_t launch_cast_bf16(const float* src, long long n, void* dst, cudaStream_t s) {
+  const long long n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  const long long cap = (long long)sm_count() * 8;
+  long long g = (n4 + 255) / 256;
+  g = g < cap ? g : cap;
+  cast_bf16_kernel<<<(unsigned)g, 256, 0, s>>>((const float4*)src, n4, (uint2*)dst);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s) {
   if (T == 0) return cudaSuccess;

@@ -6,7 +6,9 @@
 // routed to it; aiter issue 1248: g1u1 SiLU, per-token FP8; GC-MoE: fused
 // SwiGLU and requantisation):
 //   gate/up : h[r, n] = bf16( silu(G) * U ),  G = Wg[e][n] . A[r],  U = Wu[e][n] . A[r]
-//   down    : y[slot(r), n] = Wd[e][n] . h[r]
+//   down    : y[slot(r), n] = Wd[e][n] . h[r], or, fused with the combine
+//             ("Megatron" unpermute), out32[slot(r) / k, n] += w[slot(r)] * y
+//             (fp32 additions in L2, in no fixed order)
 // for every sorted row r of expert e; FP8 operands are rescaled by the
 // per-row activation scale and the per-channel weight scale after the fp32
 // accumulation.
@@ -230,8 +232,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      // L2 priorities: weights streamed once go first.  Re-read operands stay
+      // (evict-last) in the gate/up GEMM; in the down GEMM with the fused
+      // combine they are normal, so that the fp32 token rows the epilogue
+      // adds into (evict-last) stay in L2.
+      const bool keep_out = p.comb_out != nullptr;
       const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_x = keep_out ? policy_evict_normal() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       long long armed = 0;
@@ -422,23 +429,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (has1) sw1 = __ldg(p.w_scale + (long long)ti.e * p.n_out + n1);
         }
         float* o = reinterpret_cast<float*>(p.out);
+        const bool fused = p.comb_out != nullptr;
+        const uint64_t pol_out = policy_evict_last();
         for (int c = 16 * half; c < ti.nrows; c += 32) {
           float v0[16], v1[16];
-          // lanes 0..15 fetch the chunk's slots (and row scales); shuffles broadcast them
+          // lanes 0..15 fetch the chunk's slots (row scales, routing weights); shuffles broadcast them
           const bool in = lane < 16 && c + lane < ti.nrows;
           const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
           const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
+          const float wt_l = (fused && slot_l < p.n_slots) ? __ldg(p.comb_w + slot_l) : 0.f;
           tmem_ld16(tb + c, v0);
           if (has1) tmem_ld16(tb + p.tn + c, v1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int slot = __shfl_sync(0xffffffffu, slot_l, i);
             const float sa = __shfl_sync(0xffffffffu, sa_l, i);
-            if (c + i < ti.nrows) {
-              if (slot < p.n_slots) {
+            const float wt = __shfl_sync(0xffffffffu, wt_l, i);
+            if (c + i < ti.nrows && slot < p.n_slots) {
+              const float a0 = p.fp8 ? v0[i] * sa * sw0 : v0[i];
+              const float a1 = p.fp8 ? v1[i] * sa * sw1 : v1[i];
+              if (fused) {
+                // the warp's 32 lanes add to 32 consecutive floats of the token's row
+                float* orow = p.comb_out + (long long)(slot / p.k) * p.n_out;
+                red_add_f32(orow + n0, wt * a0, pol_out);
+                if (has1) red_add_f32(orow + n1, wt * a1, pol_out);
+              } else {
                 float* yr = o + (long long)slot * p.n_out;
-                yr[n0] = p.fp8 ? v0[i] * sa * sw0 : v0[i];
-                if (has1) yr[n1] = p.fp8 ? v1[i] * sa * sw1 : v1[i];
+                yr[n0] = a0;
+                if (has1) yr[n1] = a1;
               }
             }
           }

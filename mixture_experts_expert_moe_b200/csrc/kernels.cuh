@@ -55,6 +55,7 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
 cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
                               int nrows, int C, void* q, float* scale, cudaStream_t s);
 cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s);
+cudaError_t launch_cast_bf16(const float* src, long long n, void* dst, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
 
@@ -89,6 +90,8 @@ struct GemmParams {
   int32_t* status;
   long long timeout_ns;
   int* tile_counter;     // next unclaimed tile of this launch (zero at launch)
+  float* comb_out;       // down only, nullable: out32 [T, n_out] += comb_w[slot] * y instead of
+  const float* comb_w;   //   writing y (top-k combine fused into the epilogue)
 };
 
 struct GemmLaunch {
