@@ -26,6 +26,7 @@
 // wait at all.
 #include "gate.cuh"
 #include "kernels.cuh"
+#include "plan.cuh"
 
 namespace moe {
 
@@ -54,47 +55,6 @@ __device__ bool grid_wait(int* counter, int expected, long long timeout_ns) {
   }
   __syncthreads();
   return s_ok != 0;
-}
-
-// Exclusive scan of a[0..n) in shared memory by the whole CTA; returns the total.
-__device__ int block_exclusive_scan(int* a, int n) {
-  __shared__ int s_warp[32];
-  __shared__ int s_total;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthr = blockDim.x;
-  const int ipt = (n + nthr - 1) / nthr;
-  const int beg = min(n, tid * ipt), end = min(n, beg + ipt);
-  int local = 0;
-  for (int i = beg; i < end; ++i) local += a[i];
-  int incl = local;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int nw = nthr >> 5;
-    int v = lane < nw ? s_warp[lane] : 0;
-    int vi = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      int u = __shfl_up_sync(0xffffffffu, vi, off);
-      if (lane >= off) vi += u;
-    }
-    if (lane < nw) s_warp[lane] = vi - v;
-    if (lane == nw - 1) s_total = vi;
-  }
-  __syncthreads();
-  int run = s_warp[warp] + incl - local;
-  for (int i = beg; i < end; ++i) {
-    int v = a[i];
-    a[i] = run;
-    run += v;
-  }
-  __syncthreads();
-  return s_total;
 }
 
 // Issues the loads of kSub sub-steps (32 consecutive slots each) of a warp's
@@ -324,34 +284,16 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   if (kPlan && blockIdx.x == 0) {
     // ---- tile plan of the grouped GEMMs (layout in kernels.cuh) --------------
     __syncthreads();
-    int* s_pg = wcnt;              // tiles per expert -> exclusive prefix
-    int* s_pd = wcnt + E + 1;
+    int* s_g = wcnt;               // token groups per expert
+    int* sc = wcnt + E;            // 3E + 2 ints of scratch (wcnt holds 32E)
     for (int e = tid; e < E; e += blockDim.x) {
       const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
-      const int g = (rows + r.tn - 1) / r.tn;
-      r.plan[4 + e] = s_off[e];
-      r.plan[4 + E + e] = rows;
-      r.plan[4 + 2 * E + e] = g;
-      s_pg[e] = g * r.nw_gu;
-      s_pd[e] = g * r.nw_dn;
+      r.plan[plan_start(E) + e] = s_off[e];
+      r.plan[plan_rows(E) + e] = rows;
+      s_g[e] = (rows + r.tn - 1) / r.tn;
     }
     __syncthreads();
-    const int tg = block_exclusive_scan(s_pg, E);
-    const int td = block_exclusive_scan(s_pd, E);
-    for (int e = tid; e < E; e += blockDim.x) {
-      r.plan[4 + 3 * E + e] = s_pg[e];
-      r.plan[5 + 4 * E + e] = s_pd[e];
-    }
-    if (tid == 0) {
-      r.plan[4 + 4 * E] = tg;
-      r.plan[5 + 5 * E] = td;
-      r.plan[0] = tg;
-      r.plan[1] = td;
-      r.plan[plan_counter(E, true)] = 0;
-      r.plan[plan_counter(E, false)] = 0;
-      r.plan[2] = r.tn;
-      r.plan[3] = total_post;
-    }
+    finish_plan(r.plan, s_g, E, r.nw_gu, r.nw_dn, r.tn, total_post, sc);
   }
 }
 

@@ -31,6 +31,7 @@
 //   * every wait is bounded; on a timeout the CTA records MOE_DEV_TIMEOUT,
 //     drains its copies and MMAs, frees TMEM and returns.
 #include "kernels.cuh"
+#include "plan.cuh"
 
 namespace moe {
 
@@ -40,24 +41,16 @@ constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
 constexpr int kRing = 4;         // tile indices in flight from the producer to the other warps
 
-// Plan layout (int32), written by plan_kernel from the align&sort outputs.
-//   [0] tiles of the gate/up GEMM   [1] tiles of the down GEMM   [2] tn
-//   seg_start[E] @4      first sorted row of each expert
-//   seg_rows[E]  @4+E    padded rows of each expert
-//   groups[E]    @4+2E   token groups of <= tn rows
-//   pref_gu[E+1] @4+3E   exclusive prefix of gate/up tiles per expert
-//   pref_dn[E+1] @5+4E   exclusive prefix of down tiles per expert
-//   counters     @6+5E   tiles claimed so far by the gate/up and the down GEMM
-
+// Tile plan for the stand-alone FFN (moe_grouped_ffn), from the align & sort
+// outputs; layout in kernels.cuh, ordering in plan.cuh.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ expert_ids,
                                                     const int32_t* __restrict__ num_post, int P, int E, int bm,
                                                     int tn, int nw_gu, int nw_dn, int32_t* __restrict__ plan,
                                                     int32_t* status) {
   extern __shared__ int sm[];
-  int* s_first = sm;        // first block of expert
-  int* s_nblk = sm + E;     // blocks of expert
-  int* s_pg = sm + 2 * E;   // gate/up tiles -> prefix
-  int* s_pd = sm + 3 * E;   // down tiles -> prefix
+  int* s_first = sm;        // [E] first block of expert
+  int* s_nblk = sm + E;     // [E] blocks of expert -> token groups
+  int* sc = sm + 2 * E;     // [3E + 2] scratch of finish_plan
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) {
     s_first[e] = 0;
@@ -82,37 +75,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
     const int rows = s_nblk[e] * bm;
-    const int g = (rows + tn - 1) / tn;
-    plan[4 + e] = s_first[e] * bm;
-    plan[4 + E + e] = rows;
-    plan[4 + 2 * E + e] = g;
-    s_pg[e] = g * nw_gu;
-    s_pd[e] = g * nw_dn;
+    plan[plan_start(E) + e] = s_first[e] * bm;
+    plan[plan_rows(E) + e] = rows;
+    s_nblk[e] = (rows + tn - 1) / tn;
   }
   __syncthreads();
-  if (tid == 0) {  // E <= 1024: a serial scan is a few microseconds at most
-    int a = 0, b = 0;
-    for (int e = 0; e < E; ++e) {
-      plan[4 + 3 * E + e] = a;
-      plan[5 + 4 * E + e] = b;
-      a += s_pg[e];
-      b += s_pd[e];
-    }
-    plan[4 + 4 * E] = a;
-    plan[5 + 5 * E] = b;
-    plan[0] = a;
-    plan[1] = b;
-    plan[2] = tn;
-    plan[3] = np;
-    plan[plan_counter(E, true)] = 0;
-    plan[plan_counter(E, false)] = 0;
-  }
+  finish_plan(plan, s_nblk, E, nw_gu, nw_dn, tn, np, sc);
 }
 
 cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
                         int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s) {
-  plan_kernel<<<1, 1024, 4 * E * sizeof(int), s>>>(expert_ids, num_post, P, E, bm, tn, nw_gu, nw_dn, plan,
-                                                   status);
+  plan_kernel<<<1, 1024, (5 * E + 2) * sizeof(int), s>>>(expert_ids, num_post, P, E, bm, tn, nw_gu, nw_dn, plan,
+                                                         status);
   return cudaGetLastError();
 }
 
@@ -121,22 +95,36 @@ struct TileInfo {
   int e, wt, r0, nrows;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_pref, const int* s_start, const int* s_rows,
-                                                const int* s_groups, int E, int tn) {
-  int lo = 0, hi = E - 1;  // last expert whose tile range starts at or before t
+// Tile t of the list: the list position of its expert (last position whose
+// tile range starts at or before t), then weight tile and token group.
+__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_pref, const int* s_perm, const int* s_start,
+                                                const int* s_rows, const int* s_groups, int E, int tn) {
+  int lo = 0, hi = E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (s_pref[mid] <= t) lo = mid; else hi = mid - 1;
   }
   TileInfo ti;
-  ti.e = lo;
+  ti.e = s_perm[lo];
   const int local = t - s_pref[lo];
-  const int G = s_groups[lo];
+  const int G = s_groups[ti.e];
   ti.wt = local / G;
   const int g = local - ti.wt * G;
-  ti.r0 = s_start[lo] + g * tn;
-  ti.nrows = min(tn, s_rows[lo] - g * tn);
+  ti.r0 = s_start[ti.e] + g * tn;
+  ti.nrows = min(tn, s_rows[ti.e] - g * tn);
   return ti;
+}
+
+// The c-th claimed tile: hot-list tiles [0, hot) and cold-list tiles
+// [hot, n) alternate while both last, then the rest of the longer list (a
+// bijection on [0, n); claims past the end stay past the end).
+__device__ __forceinline__ int claim_to_tile(int c, int hot, int n) {
+  if (c >= n) return c;
+  const int cold = n - hot;
+  const int m = min(hot, cold);
+  if (c < 2 * m) return (c & 1) ? hot + (c >> 1) : (c >> 1);
+  const int r = c - 2 * m;
+  return hot > cold ? m + r : hot + m + r;
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, long long timeout_ns,
@@ -183,7 +171,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* s_start = s_ring + kRing + 2;
   int* s_rows = s_start + E;
   int* s_groups = s_rows + E;
-  int* s_pref = s_groups + E;   // E + 1
+  int* s_perm = s_groups + E;
+  int* s_pref = s_perm + E;     // E + 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -210,14 +199,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(s_tmem, p.tmem_cols);
     tmem_relinquish();
   }
-  const int pref_off = p.gateup ? 4 + 3 * E : 5 + 4 * E;
+  const int pref_off = plan_pref(E, p.gateup != 0);
   for (int i = threadIdx.x; i < E; i += blockDim.x) {
-    s_start[i] = p.plan[4 + i];
-    s_rows[i] = p.plan[4 + E + i];
-    s_groups[i] = p.plan[4 + 2 * E + i];
+    s_start[i] = p.plan[plan_start(E) + i];
+    s_rows[i] = p.plan[plan_rows(E) + i];
+    s_groups[i] = p.plan[plan_groups(E) + i];
+    s_perm[i] = p.plan[plan_perm(E) + i];
   }
   for (int i = threadIdx.x; i <= E; i += blockDim.x) s_pref[i] = p.plan[pref_off + i];
-  const int n_tiles = p.plan[p.gateup ? 0 : 1];
+  const int n_tiles = p.plan[p.gateup ? PLAN_TILES_GU : PLAN_TILES_DN];
+  const int n_hot = p.plan[p.gateup ? PLAN_HOT_GU : PLAN_HOT_DN];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -250,11 +241,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
-        const int t = atomicAdd(p.tile_counter, 1);
+        const int t = claim_to_tile(atomicAdd(p.tile_counter, 1), n_hot, n_tiles);
         s_ring[slot] = t;
         mbar_arrive(&t_full[slot]);
         if (t >= n_tiles) break;
-        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+        const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
         int row0, row1;
         bool has1 = true;
         if (p.gateup) {
@@ -318,7 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int t = s_ring[slot];
         mbar_arrive(&t_empty[slot]);
         if (t >= n_tiles) break;
-        const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+        const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
         const bool has1 = p.gateup || ti.wt * 2 * kWRows + kWRows < p.n_out;
         const int acc = it % p.n_acc;
         const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
@@ -383,7 +374,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[slot]);
       if (t >= n_tiles) break;
-      const TileInfo ti = decode_tile(t, s_pref, s_start, s_rows, s_groups, E, p.tn);
+      const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
       const int acc = it % p.n_acc;
       const uint32_t acc_phase = (uint32_t)(it / p.n_acc) & 1u;
       if (!wait_or_abort(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag)) break;
@@ -516,7 +507,7 @@ size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
   const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
   (void)gateup;
   return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5 + 2 * kRing) * 8 + (kRing + 4) * 4 +
-         (size_t)(4 * E + 1) * 4;
+         (size_t)(5 * E + 1) * 4;
 }
 
 int gemm_pick_stages(int gateup, int tn, int E) {
