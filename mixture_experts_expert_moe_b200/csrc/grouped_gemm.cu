@@ -19,9 +19,13 @@
 //     (16..256).  An expert's weight tile is streamed once for up to 256 of
 //     its tokens, so weight traffic does not grow with the block size (the
 //     lesson of the aiter issue's I/O table).
-//   * persistent CTAs, one per SM, walk a device-built tile list ordered
-//     expert -> weight tile -> token group, so CTAs that run at the same
-//     time share weight tiles through L2 when an expert has several groups.
+//   * persistent CTAs, one per SM, claim tiles from a global counter over a
+//     device-built tile list ordered expert -> weight tile -> token group
+//     (experts with several groups first, claims alternating between them
+//     and the others; see plan.cuh), so CTAs that run at the same time share
+//     weight tiles through L2 when an expert has several groups.  The TMA
+//     warp claims; a 4-entry shared-memory ring hands the index to the MMA
+//     and epilogue warps.
 //   * warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread)
 //     and owns the TMEM allocation, warps 2..9 drain TMEM (tcgen05.ld, two
 //     warps per lane quarter on alternate column chunks) and run the
