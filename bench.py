@@ -146,6 +146,23 @@ def touched_experts(layer, d):
     return int(torch.unique(ids).numel()), ids
 
 
+def max_over_ranks(value, device):
+    """The largest of every rank's value (the value itself in a one-process
+    run); every rank must call it, in the same order."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, steps, ms):
+    """Whole-job units/s of `world` replicas that each process `units_per_rank`
+    units per step, `steps` steps in `ms` milliseconds (the max over ranks)."""
+    return world * units_per_rank * steps / (ms * 1e-3)
+
+
 def kernels_per_step(cfg, out_dtype):
     """Kernels of this library one moe_forward launches: the routing kernel
     (gate + align + plan), the gather, the gate/up and down GEMMs and the
@@ -401,11 +418,7 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
     used_graph = graph is not None
     del graph
     step_ms = ms / args.steps
@@ -423,14 +436,18 @@ def run_ours(args):
                 "traffic": traffic_for(f"grouped_gemm_{dom}", workload_name(cfg, "bf16")),
                 "kernel": f"grouped_gemm_kernel ({dom} projection)", "launch_ms": stages[dom],
                 "algorithmic_bytes": kbytes, "peak_source": f"{pk_src} hbm_gbs (copy)"}
-    ems, h2d, d2h = time_e2e(cfg, layer, d, max(10, args.steps // 2), 3)
-    e2e = {"value": world * cfg.T * max(10, args.steps // 2) / (ems * 1e-3), "unit": "tokens/s",
+    e2e_steps = max(10, args.steps // 2)
+    if world > 1:
+        torch.distributed.barrier()
+    ems, h2d, d2h = time_e2e(cfg, layer, d, e2e_steps, 3)
+    ems = max_over_ranks(ems, dev)
+    e2e = {"value": job_throughput(world, cfg.T, e2e_steps, ems), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del layer, d
     torch.cuda.empty_cache()
 
     extra = {}
-    if rank == 0 and not args.quick:
+    if world == 1 and not args.quick:   # single-GPU reports (other ranks would idle in a barrier)
         extra["a8w8"], _, _ = layer_report(m, cfg.with_(a8w8=True), 50, 5, dev, pk, "a8w8")
         extra["mixtral"], _, _ = layer_report(m, CONFIGS["mixtral"], 20, 3, dev, pk, "bf16")
         extra["deepseek_shared"], _, _ = layer_report(m, CONFIGS["deepseek_shared"], 50, 5, dev, pk, "bf16")
@@ -449,7 +466,7 @@ def run_ours(args):
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": world * cfg.T * args.steps / (ms * 1e-3), "unit": "tokens/s",
+        "metric": METRIC, "value": job_throughput(world, cfg.T, args.steps, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) random-init expert weights)",
