@@ -24,6 +24,8 @@
 // with gating in front and the GEMM tile plan behind, is the single routing
 // launch of moe_forward; with one CTA (small batches) it needs no grid-wide
 // wait at all.
+#include <atomic>
+
 #include "gate.cuh"
 #include "kernels.cuh"
 #include "plan.cuh"
@@ -343,14 +345,18 @@ cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cu
 // with the grid).  The function attribute and occupancy are set up once per
 // device (they depend only on the device and the kernel).
 int align_max_ctas(int E, int* err_out) {
-  static int cached_sms[64] = {0};
-  static int cached_smem[64] = {0};
+  // per device: SM count once the attribute and occupancy check succeeded
+  // (atomic: host threads may race here; they all store the same value)
+  static std::atomic<int> cached_sms[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   *err_out = (int)e;
   if (e != cudaSuccess) return 0;
   const int need = (int)align_smem_bytes(1024);
-  if (dev < 64 && cached_sms[dev] > 0 && cached_smem[dev] >= need) return cached_sms[dev];
+  if (dev < 64) {
+    const int c = cached_sms[dev].load(std::memory_order_acquire);
+    if (c > 0) return c;
+  }
   int sms = 0, per_sm = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
@@ -360,10 +366,7 @@ int align_max_ctas(int E, int* err_out) {
   *err_out = (int)e;
   if (e != cudaSuccess || per_sm < 1) return 0;
   (void)E;
-  if (dev < 64) {
-    cached_sms[dev] = sms;
-    cached_smem[dev] = need;
-  }
+  if (dev < 64) cached_sms[dev].store(sms, std::memory_order_release);
   return sms;
 }
 

@@ -21,53 +21,67 @@
 
 namespace moe {
 
+// Order-preserving map of a finite float to uint32: a > b iff key(a) > key(b),
+// and a == b (as floats) iff key(a) == key(b), so -0 maps like +0.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  const uint32_t b = f == 0.f ? 0u : __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 template <int EPL>
 __device__ __forceinline__ void gate_token(const float* __restrict__ logits, const float* __restrict__ bias,
                                            bool select_only, long long t, int E, int k, int n_shared,
                                            int32_t* __restrict__ ids, float* __restrict__ w, int lane) {
-  float v[EPL], raw[EPL], b[EPL];
-  // all loads first, then the adds (a use right after a load would serialise them)
+  float v[EPL];
+  {
+    float b[EPL];
+    // all loads first, then the adds (a use right after a load would serialise them)
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = lane + 32 * j;
-    raw[j] = e < E ? __ldg(logits + t * E + e) : -FLT_MAX;
-    b[j] = (bias && e < E) ? __ldg(bias + e) : 0.f;
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = e < E ? __ldg(logits + t * E + e) : -FLT_MAX;
+      b[j] = (bias && e < E) ? __ldg(bias + e) : 0.f;
+    }
+    if (bias) {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (lane + 32 * j < E) v[j] = __fadd_rn(v[j], b[j]);
+    }
   }
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) v[j] = (bias && lane + 32 * j < E) ? __fadd_rn(raw[j], b[j]) : raw[j];
+  // Each round: the lane's best untaken score (first one on equal scores, so
+  // the lowest expert index), a warp max of its order-preserving 32-bit key
+  // (redux.sync), then a warp min of the expert index among the lanes that
+  // hold that key (ties go to the lower index).  The winner's score is the
+  // key inverted.
   uint32_t taken = 0;
-  float my_val = 0.f, my_raw = 0.f;
+  float my_val = 0.f;
   int my_id = 0;
   for (int r = 0; r < k; ++r) {
-    float best = -FLT_MAX, braw = 0.f;
+    uint32_t bkey = 0u;          // below every finite score's key
     int be = INT_MAX;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && (be == INT_MAX || v[j] > best)) {
-        best = v[j];
-        braw = raw[j];
+      const uint32_t key = score_key(v[j]);
+      if (e < E && !((taken >> j) & 1u) && (be == INT_MAX || key > bkey)) {
+        bkey = key;
         be = e;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const float oraw = __shfl_xor_sync(0xffffffffu, braw, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (oe != INT_MAX && (be == INT_MAX || ob > best || (ob == best && oe < be))) {
-        best = ob;
-        braw = oraw;
-        be = oe;
-      }
-    }
-    if (lane == (be & 31)) taken |= 1u << (be >> 5);
+    const uint32_t wkey = __reduce_max_sync(0xffffffffu, bkey);
+    const int win = (int)__reduce_min_sync(0xffffffffu, (be != INT_MAX && bkey == wkey) ? (uint32_t)be : 0xffffffffu);
+    if (lane == (win & 31)) taken |= 1u << (win >> 5);
     if (lane == r) {
-      my_val = best;
-      my_raw = braw;
-      my_id = be;
+      my_val = key_score(wkey);
+      my_id = win;
     }
   }
+  // selection-only bias: the weights use the chosen experts' raw logits
+  float my_raw = my_val;
+  if (select_only && bias && lane < k) my_raw = __ldg(logits + t * E + my_id);
   const float l = lane < k ? (select_only ? my_raw : my_val) : -FLT_MAX;
   float top = l;
 #pragma unroll
