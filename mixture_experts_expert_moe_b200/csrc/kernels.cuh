@@ -52,8 +52,11 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
 // per-row E4M3 quantisation of bf16 rows of length C; rows = *nrows_dev if
 // non-null, else nrows.  With `sorted`, output row r quantises source row
 // sorted[r] / k (zero codes, scale 1 for padding slots >= N).
+// rows [0, *nrows_dev) (or [0, nrows) when nrows_dev is null; nrows bounds
+// *nrows_dev) of src [.., C] bf16 -> E4M3 codes + fp32 scales; with sorted,
+// row r quantises token sorted[r] / k (zero codes, scale 1 for padding)
 cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
-                              int nrows, int C, void* q, float* scale, cudaStream_t s);
+                              int nrows, int C, void* q, float* scale, int32_t* status, cudaStream_t s);
 cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s);
 cudaError_t launch_cast_bf16(const float* src, long long n, void* dst, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
