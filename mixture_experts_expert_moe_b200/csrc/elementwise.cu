@@ -88,8 +88,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 // GC-MoE: requantisation between the GEMMs).  s = amax / 448 in fp32 (1 for
 // an all-zero row); code = e4m3_rne_satfinite(v / s) with v / s the correctly
 // rounded fp32 quotient.  One warp per row with the row held in registers (VPL
-// 16-byte vectors of 8 bf16 per lane); longer rows take one CTA per row (up
-// to 256*16*8 elements), beyond that two passes.  With a row map the kernel also gathers (sorted row r quantises its
+// 16-byte vectors of 8 bf16 per lane) below 4096 elements; longer rows are
+// staged in shared memory by bulk copies (quant_rows_bulk_kernel), and rows
+// too long for that (over 100K elements) take two passes.  With a row map the kernel also gathers (sorted row r quantises its
 // token).
 //
 // The quotient comes from one reciprocal per row and a correction step per
@@ -295,50 +296,7 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
-// Long rows (up to 256*16*8 elements): one CTA of 256 threads per row, the row
-// held in registers (VPT 16-byte vectors per thread), a block-wide amax, one
-// read of the row.
-template <int VPT>
-__global__ void __launch_bounds__(256) quant_rows_block_kernel(const uint4* __restrict__ src,
-                                                               const int32_t* __restrict__ sorted, int N, int k,
-                                                               const int32_t* __restrict__ nrows_dev, int nrows,
-                                                               int vec, uint2* __restrict__ q,
-                                                               float* __restrict__ scale) {
-  __shared__ float s_amax[8];
-  const int n = nrows_dev ? *nrows_dev : nrows;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r = blockIdx.x; r < n; r += gridDim.x) {
-    const long long sr = quant_src_row(sorted, r, N, k);
-    uint2* dst = q + (long long)r * vec;
-    if (sr < 0) {
-      for (int c = threadIdx.x; c < vec; c += 256) dst[c] = make_uint2(0, 0);
-      if (threadIdx.x == 0) scale[r] = 1.f;
-      continue;
-    }
-    const uint4* row = src + sr * vec;
-    uint4 v[VPT];
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int c = threadIdx.x + 256 * i;
-      v[i] = c < vec ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
-      amax = fmaxf(amax, absmax8(v[i]));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) s_amax[warp] = amax;
-    __syncthreads();
-    amax = s_amax[lane & 7];
-#pragma unroll
-    for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    __syncthreads();   // s_amax is rewritten by the next row
-    const RowScale rs = row_scale(amax);
-    quant_store<VPT>(v, rs, dst, threadIdx.x, 256, vec);
-    if (threadIdx.x == 0) scale[r] = rs.s;
-  }
-}
-
-// Rows longer than the register-resident limits: one warp per row, two passes
+// Rows too long to stage (over 100K elements): one warp per row, two passes
 
 // (the second pass re-reads the row from L1/L2).
 __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __restrict__ src,
@@ -431,17 +389,7 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int
   else if (vpl <= 4) MOE_QUANT(4);
   else if (vpl <= 8) MOE_QUANT(8);
   else if (vpl <= 16) MOE_QUANT(16);
-  else {
-    const int vpt = (vec + 255) / 256;
-    const long long cap = (long long)sm_count() * 8;
-    const int gb = (int)(nrows < 1 ? 1 : (nrows < cap ? nrows : cap));
-#define MOE_QUANT_B(V) quant_rows_block_kernel<V><<<gb, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale)
-    if (vpt <= 4) MOE_QUANT_B(4);
-    else if (vpt <= 8) MOE_QUANT_B(8);
-    else if (vpt <= 16) MOE_QUANT_B(16);
-    else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
-#undef MOE_QUANT_B
-  }
+  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
 #undef MOE_QUANT
   return cudaGetLastError();
 }
