@@ -72,7 +72,10 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2 } moe_dtype_t;
 MOE_API const char* moe_status_string(int status);
 /* Text of the last CUDA error seen by this thread inside the library. */
 MOE_API const char* moe_last_cuda_error(void);
-/* ABI version (major*100 + minor). */
+/* ABI version (major*100 + minor); equals MOE_ABI_VERSION of the header the
+ * library was built with.  Major 2: moe_topk_gate takes bias_mode and
+ * n_shared, moe_forward_args ends with n_shared and bias_mode. */
+#define MOE_ABI_VERSION 200
 MOE_API int moe_version(void);
 
 /* ---------------------------------------------------------------------------

@@ -47,6 +47,7 @@ class ForwardArgs(ctypes.Structure):
 
 
 MOE_BIAS_LOGITS, MOE_BIAS_SELECT = 0, 1
+ABI_VERSION = 200   # MOE_ABI_VERSION of include/moe_b200.h
 _BIAS_MODES = {"logits": MOE_BIAS_LOGITS, "select": MOE_BIAS_SELECT}
 
 
@@ -82,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+        if lib.moe_version() != ABI_VERSION:
+            raise ImportError(f"{path} implements ABI {lib.moe_version()}, this binding expects {ABI_VERSION}: "
+                              "rebuild it with `python -m mixture_experts_expert_moe_b200.build_lib`")
         _LIB = lib
     return _LIB
 

@@ -348,7 +348,7 @@ const char* moe_status_string(int s) {
 
 const char* moe_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
-int moe_version(void) { return 100; }
+int moe_version(void) { return MOE_ABI_VERSION; }
 
 moe_status_t moe_topk_gate(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
                            int n_shared, int32_t* topk_ids, float* topk_w, void* stream) {

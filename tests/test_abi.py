@@ -31,7 +31,7 @@ def test_status_strings_and_version():
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
     assert lib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
-    assert lib.moe_version() == 100
+    assert lib.moe_version() == m.ABI_VERSION == 200
 
 
 def test_align_sizes():
