@@ -24,7 +24,7 @@ Sources (page title, section):
 * [GC] GC-MoE abstract (zhuanzhiai.com): fused SwiGLU with requantisation
   between the two grouped GEMMs.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the same list is kept with the design notes):
 
 1. Top-k ties go to the lower expert index; ids are listed by descending
    logit.  Weights are the softmax over all E logits, renormalised over the
