@@ -46,13 +46,18 @@ Readings where the pages are silent (the same list is kept with the design notes
    fp32-accumulated reference the tolerances are quoted against).
 
 Pins (tests/test_oracle_*.py): brute-force top-k over all subsets; the k=E
-case equals a library softmax; brute-force align via Python ``sorted``;
-align invariants; bf16 rounding equals torch's fp32->bf16 cast; the e4m3
-codec round-trips all 256 codes, matches torch's e4m3 cast in range and
-saturates beyond; identical experts reproduce a dense SwiGLU FFN computed
-with library matmuls; k=1 forced routing reproduces the dense FFN; x=0 gives
-0; token permutation equivariance; expert relabelling invariance; FP8 with
-exactly representable operands equals the unquantised product.
+case equals a library softmax; both bias modes against brute-force selection
+on logit + bias with library-softmax weights (of the biased or the raw
+logits), a constant bias and a bias that forces a set of experts;
+brute-force align via Python ``sorted``; align invariants; bf16 rounding
+equals torch's fp32->bf16 cast; the e4m3 codec round-trips all 256 codes,
+matches torch's e4m3 cast in range and saturates beyond; identical experts
+reproduce a dense SwiGLU FFN computed with library matmuls; k=1 forced
+routing reproduces the dense FFN; shared experts add exactly their dense
+FFNs (the layer with them minus the layer without them; routed outputs
+forced to zero); x=0 gives 0; token permutation equivariance; expert
+relabelling invariance; FP8 with exactly representable operands equals the
+unquantised product.
 """
 from __future__ import annotations
 
