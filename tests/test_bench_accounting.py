@@ -1,0 +1,53 @@
+"""bench.py's accounting, checked by hand on small numbers (CPU).
+
+The roofline objects divide these byte and FLOP counts by measured times, so
+a wrong count would silently scale every reported fraction.
+"""
+import os
+import sys
+
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from moe_inputs import CONFIGS, MoEConfig  # noqa: E402
+
+
+def test_slot_pairs_count_shared_experts():
+    assert bench.slot_pairs(MoEConfig("t", T=10, H=128, I=128, E=8, k=2, bm=16)) == 20
+    assert bench.slot_pairs(MoEConfig("t", T=10, H=128, I=128, E=8, k=2, bm=16, n_shared=1)) == 30
+
+
+def test_kernels_per_step():
+    bf16 = MoEConfig("t", T=2048, H=128, I=128, E=256, k=8, bm=64)
+    assert bench.kernels_per_step(bf16, None) == 5            # route, gather, gate/up, down, combine/round
+    assert bench.kernels_per_step(bf16.with_(a8w8=True), None) == 7   # + quant (16384 slots > 4096) + requant
+    assert bench.kernels_per_step(bf16.with_(T=16, a8w8=True), None) == 6   # fused quant + gather
+
+
+def test_gateup_and_down_bytes_by_hand():
+    cfg = MoEConfig("t", T=4, H=256, I=128, E=8, k=2, bm=16)
+    touched = 3
+    # bf16: 3 experts x (2*128*256 weights x 2 B) + 8 pairs x 256 x 2 B (rows) + 8 pairs x 128 x 2 B (h)
+    assert bench.gateup_bytes(cfg, touched) == 3 * 2 * 128 * 256 * 2 + 8 * 256 * 2 + 8 * 128 * 2
+    # down: 3 x 256*128 x 2 + 8 x 128 x 2 (h) + 8 x 256 x 4 (fp32 y rows)
+    assert bench.down_bytes(cfg, touched) == 3 * 256 * 128 * 2 + 8 * 128 * 2 + 8 * 256 * 4
+    a8 = cfg.with_(a8w8=True)
+    # E4M3 weights + fp32 per-channel scales
+    assert bench.gateup_bytes(a8, touched) == 3 * (2 * 128 * 256 + 8 * 128) + 8 * 256 + 8 * 128 * 2
+
+
+def test_headline_workload_name():
+    name = bench.workload_name(CONFIGS["deepseek"], "bf16")
+    assert name == "deepseek_bf16: T=2048 H=7168 I=2048 E=256 k=8 bm=64"
+    assert bench.workload_name(CONFIGS["deepseek_shared"], "bf16").endswith("+bias(selection only) +1 shared")
+
+
+def test_traffic_lookup_needs_matching_source():
+    # the committed table is keyed by the kernel source hash: a made-up workload has no entry
+    assert bench.traffic_for("grouped_gemm_gateup", "no such workload") is None
+
+
+@pytest.mark.parametrize("world,units,steps,ms", [(1, 2048, 100, 400.0), (8, 2048, 50, 210.0)])
+def test_job_throughput(world, units, steps, ms):
+    assert bench.job_throughput(world, units, steps, ms) == pytest.approx(world * units * steps / (ms / 1000))
