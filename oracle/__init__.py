@@ -11,7 +11,9 @@ arithmetic.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against brute force,
 closed forms, library routines and the figures the pages print.  See the
-module docstring of :mod:`oracle.moe_oracle` for the list of pins.
+module docstrings of :mod:`oracle.moe_oracle` (the layer forward) and
+:mod:`oracle.mx_oracle` (MX block-scaled operands, the next FFN variant) for
+the lists of pins.
 """
 from .moe_oracle import (  # noqa: F401
     bf16_round,
