@@ -58,7 +58,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2,   /* valid but not handled (e.g. H % 128 != 0)   */
   MOE_ERR_WORKSPACE = 3,     /* workspace smaller than the size query says  */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (see moe_last_cuda_error) */
-  MOE_ERR_DEVICE = 5         /* no sm_100 device current                    */
+  MOE_ERR_DEVICE = 5         /* no sm_100 device: none current, no GPU or
+                                driver at all, or another architecture      */
 } moe_status_t;
 
 typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2 } moe_dtype_t;

@@ -44,6 +44,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 moe_status_t check_device() {
   int dev = 0, major = 0;
   cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) {
+    cuda_fail(e, "cudaGetDevice");   // keeps the text for moe_last_cuda_error
+    return MOE_ERR_DEVICE;           // no usable GPU at all: there is no CPU fallback
+  }
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");

@@ -77,7 +77,9 @@ extern "C" MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, 
   if (E > moe::kNoallocMaxExperts) return MOE_ERR_UNSUPPORTED;  // beyond the built-in scratch
 
   int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge == cudaErrorNoDevice || ge == cudaErrorInsufficientDriver) return MOE_ERR_DEVICE;
+  if (ge != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (major != 10) return MOE_ERR_DEVICE;
 

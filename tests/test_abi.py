@@ -108,3 +108,83 @@ def test_forward_workspace_and_validation():
     assert lib.moe_forward(ctypes.byref(a), None, 0, None, None) == 1
     assert lib.moe_combine(None, None, 4, 2, 6, None, 0, None) == 1    # H % 4
     assert lib.moe_combine(None, None, 4, 2, 8, None, 5, None) == 1    # dtype
+
+
+# ---------------------------------------------------------------------------
+# argument errors are reported before anything touches the device
+# ---------------------------------------------------------------------------
+_HOST = (ctypes.c_uint8 * 4096)()          # a 16-byte-aligned host block used only as a non-null address
+_ADDR = (ctypes.addressof(_HOST) + 15) // 16 * 16
+
+
+def _fwd(**kw):
+    a = dict(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, out_dtype=0, x=_ADDR, logits=_ADDR,
+             w13=_ADDR, w2=_ADDR, out=_ADDR)
+    a.update(kw)
+    return m.ForwardArgs(**a)
+
+
+def test_forward_rejects_misaligned_and_missing_scales():
+    lib = m.load_library()
+    for bad in (dict(x=_ADDR + 2), dict(w13=_ADDR + 8), dict(out=_ADDR + 4)):
+        assert lib.moe_forward(ctypes.byref(_fwd(**bad)), ctypes.c_void_p(_ADDR), 1 << 40, None, None) == 1
+    # FP8 weights need their scales
+    assert lib.moe_forward(ctypes.byref(_fwd(wdtype=1)), ctypes.c_void_p(_ADDR), 1 << 40, None, None) == 1
+    # a misaligned workspace
+    assert lib.moe_forward(ctypes.byref(_fwd()), ctypes.c_void_p(_ADDR + 1), 1 << 40, None, None) == 1
+
+
+def test_forward_workspace_too_small():
+    lib = m.load_library()
+    a = _fwd()
+    n = ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert lib.moe_forward(ctypes.byref(a), ctypes.c_void_p(_ADDR), n.value - 1, None, None) == 3
+
+
+def test_forward_without_a_device_fails_loudly():
+    """Valid arguments on a machine without an sm_100 device: MOE_ERR_DEVICE
+    (there is no CPU fallback)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    lib = m.load_library()
+    a = _fwd()
+    n = ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert lib.moe_forward(ctypes.byref(a), ctypes.c_void_p(_ADDR), n.value, None, None) == 5
+
+
+def test_forward_with_no_tokens_is_a_no_op():
+    lib = m.load_library()
+    assert lib.moe_forward(ctypes.byref(_fwd(T=0)), None, 0, None, None) == 0
+
+
+def test_gate_with_no_tokens_is_a_no_op():
+    lib = m.load_library()
+    assert lib.moe_topk_gate(None, None, 0, 0, 8, 2, 0, None, None, None) == 0
+
+
+def test_ffn_rejects_small_workspace_and_missing_scales():
+    lib = m.load_library()
+    a = _ffn(x=_ADDR, w13=_ADDR, w2=_ADDR, sorted_ids=_ADDR, expert_ids=_ADDR, num_post=_ADDR)
+    n = ctypes.c_size_t()
+    assert lib.moe_ffn_workspace(ctypes.byref(a), ctypes.byref(n)) == 0
+    y = ctypes.c_void_p(_ADDR)
+    assert lib.moe_grouped_ffn(ctypes.byref(a), y, ctypes.c_void_p(_ADDR), n.value - 16, None, None) == 3
+    a8 = _ffn(wdtype=1, x=_ADDR, w13=_ADDR, w2=_ADDR, sorted_ids=_ADDR, expert_ids=_ADDR, num_post=_ADDR)
+    assert lib.moe_grouped_ffn(ctypes.byref(a8), y, ctypes.c_void_p(_ADDR), 1 << 40, None, None) == 1
+
+
+def test_align_sort_argument_errors():
+    lib = m.load_library()
+    p = ctypes.c_void_p(_ADDR)
+    # outputs missing
+    assert lib.moe_align_sort(p, 16, 2, 8, 16, None, p, p, p, 1 << 20, None, None) == 1
+    # workspace below moe_align_sort_sizes' figure
+    ws = ctypes.c_size_t()
+    assert lib.moe_align_sort_sizes(16, 2, 8, 16, None, None, ctypes.byref(ws)) == 0
+    assert lib.moe_align_sort(p, 16, 2, 8, 16, p, p, p, p, ws.value - 1, None, None) == 3
+    # the no-allocation variant: more experts than its built-in scratch holds
+    assert lib.moe_align_sort_noalloc(p, 16, 2, 257, 16, p, p, p, None, None) == 2
+    assert lib.moe_align_sort_noalloc(p, 16, 2, 8, 16, None, p, p, None, None) == 1
