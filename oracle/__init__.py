@@ -12,8 +12,9 @@ arithmetic.
 Every function is pinned by ``tests/test_oracle_*.py`` against brute force,
 closed forms, library routines and the figures the pages print.  See the
 module docstrings of :mod:`oracle.moe_oracle` (the layer forward) and
-:mod:`oracle.mx_oracle` (MX block-scaled operands, the next FFN variant) for
-the lists of pins.
+:mod:`oracle.mx_oracle` (MX block-scaled operands, the next FFN variant) and
+:mod:`oracle.backward_oracle` (the layer's backward pass) for the lists of
+pins.
 """
 from .moe_oracle import (  # noqa: F401
     bf16_round,
