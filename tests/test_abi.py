@@ -188,3 +188,24 @@ def test_align_sort_argument_errors():
     # the no-allocation variant: more experts than its built-in scratch holds
     assert lib.moe_align_sort_noalloc(p, 16, 2, 257, 16, p, p, p, None, None) == 2
     assert lib.moe_align_sort_noalloc(p, 16, 2, 8, 16, None, p, p, None, None) == 1
+
+
+def _fwd_ws(**kw):
+    lib = m.load_library()
+    a = dict(T=64, H=256, I=128, E=8, k=2, block_size=16, wdtype=0, out_dtype=0)
+    a.update(kw)
+    n = ctypes.c_size_t()
+    assert lib.moe_forward_workspace(ctypes.byref(m.ForwardArgs(**a)), ctypes.byref(n)) == 0
+    return n.value
+
+
+def test_forward_workspace_follows_the_combine_rule():
+    """k + n_shared >= 4: the combine is fused, the workspace holds an fp32
+    token accumulator [T, H] only for bf16 output (an f32 output is the
+    accumulator).  Fewer slots: per-slot rows [T*k, H] for either output."""
+    T, H = 64, 256
+    fused_bf16, fused_f32 = _fwd_ws(k=4, out_dtype=0), _fwd_ws(k=4, out_dtype=2)
+    assert fused_bf16 - fused_f32 == T * H * 4
+    assert _fwd_ws(k=2, out_dtype=0) == _fwd_ws(k=2, out_dtype=2)
+    # a shared expert counts as a slot: k = 3 + 1 shared is fused as well
+    assert _fwd_ws(k=3, n_shared=1, out_dtype=0) - _fwd_ws(k=3, n_shared=1, out_dtype=2) == T * H * 4
