@@ -109,6 +109,26 @@ def fp8_weights(E, rows, cols, std, seed, device="cpu"):
     return codes, scales
 
 
+def mx_weights(E, rows, cols, elem, seed, scale_code_mean=122):
+    """MX block-scaled weights drawn directly (no quantisation step): uint8
+    element codes [E, rows, cols] uniform over the finite codes of `elem`
+    ("e2m1": 4-bit codes 0..15; "e4m3": the E4M3FN codes except NaN), and
+    E8M0 scale codes [E, rows, cols/32] = scale_code_mean + {-1, 0, +1}
+    (powers of two around 2^(mean-127))."""
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    rng = np.random.default_rng(seed)
+    if elem == "e2m1":
+        codes = rng.integers(0, 16, size=(E, rows, cols), dtype=np.uint8)
+    elif elem == "e4m3":
+        codes = rng.integers(0, 255, size=(E, rows, cols), dtype=np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0          # no NaN codes
+    else:
+        raise ValueError(elem)
+    scales = (scale_code_mean + rng.integers(-1, 2, size=(E, rows, cols // 32))).astype(np.uint8)
+    return codes, scales
+
+
 def make_layer(cfg: MoEConfig, device="cpu", weights=True):
     """All inputs of one MoE layer forward for ``cfg``.
 

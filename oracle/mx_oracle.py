@@ -47,7 +47,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .moe_oracle import _silu, bf16_round, e4m3_decode, e4m3_encode
+from .moe_oracle import _silu, add_shared, bf16_round, combine, e4m3_decode, e4m3_encode, topk_gate
 
 MX_BLOCK = 32
 
@@ -184,6 +184,20 @@ def ffn_mx(x, ids, w13_codes, w13_scales, w2_codes, w2_scales, w_elem: str = "e2
     return y
 
 
+def moe_forward_mx(x, logits, k, w13_codes, w13_scales, w2_codes, w2_scales, w_elem="e2m1", bias=None,
+                   bias_mode="logits", n_shared=0, tokens=None):
+    """Gate -> MX expert FFN -> combine (the layer of ``moe_oracle.moe_forward``
+    with MX operands).  Returns (out float64, ids, weights)."""
+    ids, w = topk_gate(logits, k, bias, bias_mode)
+    if n_shared:
+        ids, w = add_shared(ids, w, np.asarray(logits).shape[1], n_shared)
+    T, kk = ids.shape
+    toks = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    slots = (toks[:, None] * kk + np.arange(kk)[None, :]).reshape(-1)
+    y = ffn_mx(x, ids, w13_codes, w13_scales, w2_codes, w2_scales, w_elem=w_elem, slots=slots)
+    return combine(y, w[toks]), ids, w
+
+
 __all__ = ["MX_BLOCK", "e2m1_decode", "e2m1_values", "e2m1_encode", "e8m0_decode", "mx_quantize",
-           "mx_dequantize", "mx_dot_blocks", "ffn_mx"]
+           "mx_dequantize", "mx_dot_blocks", "ffn_mx", "moe_forward_mx"]
 

@@ -138,3 +138,32 @@ def test_mx_ffn_identical_experts_is_dense(w_elem):
     hq = torch.from_numpy(mx.mx_dequantize(*mx.mx_quantize(h, "e4m3"), "e4m3"))
     dense = (hq @ torch.from_numpy(mx.mx_dequantize(c2, s2, w_elem)).T).numpy()
     np.testing.assert_allclose(y, np.repeat(dense, k, axis=0), rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("w_elem", ["e2m1", "e4m3"])
+def test_mx_layer_with_identical_experts_is_dense(w_elem):
+    """Layer level: routing and the combine of MX expert outputs; with every
+    expert (routed and shared) identical, out = (sum of the token's weights)
+    x the dense FFN, and the routed weights sum to 1."""
+    from moe_inputs import mx_weights
+    rng = np.random.default_rng(8)
+    T, H, I, E, k, S = 10, 64, 32, 6, 2, 1
+    x = mo.bf16_round(rng.standard_normal((T, H)))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    c13, s13 = mx_weights(1, 2 * I, H, w_elem, seed=1)
+    c2, s2 = mx_weights(1, H, I, w_elem, seed=2)
+    out, ids, w = mx.moe_forward_mx(x, logits, k, [c13[0]] * (E + S), [s13[0]] * (E + S), [c2[0]] * (E + S),
+                                    [s2[0]] * (E + S), w_elem=w_elem, n_shared=S)
+    y1 = mx.ffn_mx(x, np.zeros((T, 1), np.int32), [c13[0]], [s13[0]], [c2[0]], [s2[0]], w_elem=w_elem)
+    np.testing.assert_allclose(w[:, :k].astype(np.float64).sum(1), 1.0, atol=1e-6)
+    np.testing.assert_allclose(out, y1 * w.astype(np.float64).sum(1, keepdims=True), rtol=1e-9, atol=1e-12)
+
+
+def test_mx_weight_generator_codes_and_scales():
+    from moe_inputs import mx_weights
+    c, s = mx_weights(2, 8, 64, "e4m3", seed=3)
+    assert c.shape == (2, 8, 64) and s.shape == (2, 8, 2)
+    assert not np.any((c & 0x7F) == 0x7F)                 # no NaN codes
+    assert set(np.unique(s)) <= {121, 122, 123}
+    c4, _ = mx_weights(1, 4, 32, "e2m1", seed=4)
+    assert c4.max() <= 15
