@@ -68,6 +68,11 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2 } moe_dtype_t;
 #define MOE_DEV_BAD_EXPERT_ID 0x1  /* an expert id outside [0, E): slot skipped */
 #define MOE_DEV_TIMEOUT       0x2  /* a bounded wait ran out; outputs unspecified */
 #define MOE_DEV_BAD_PLAN      0x4  /* routing metadata inconsistent with sizes  */
+#define MOE_DEV_DRAIN_TIMEOUT 0x8  /* after a timeout, a GEMM CTA also gave up
+                                      waiting for its own copies or MMAs in
+                                      flight before freeing its tensor memory:
+                                      the device state is undefined; do not call
+                                      the library again in this CUDA context    */
 
 /* Human-readable name of a status code.  Host only; never fails. */
 MOE_API const char* moe_status_string(int status);
@@ -149,9 +154,13 @@ MOE_API moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int k, int E
  * held by every GPU that loads the library until the process exits).
  * Limit: E <= MOE_NOALLOC_MAX_EXPERTS, otherwise MOE_ERR_UNSUPPORTED and
  * nothing is launched.  The first call on a device looks up the array's
- * device address (make that call before any stream capture).  All calls
- * share the array: calls that overlap on the GPU race; order them on one
- * stream.  Allocates nothing.
+ * device address and keeps it per device ordinal (make that call before any
+ * stream capture).  The kept address belongs to the device's primary context,
+ * the one the CUDA runtime uses by default: do not call this entry point from
+ * another context of the device, nor after cudaDeviceReset on it (the address
+ * would then name memory that is gone).  All calls share the array: calls
+ * that overlap on the GPU race; order them on one stream.  Allocates nothing.
+ * CUDA failures return MOE_ERR_CUDA with the text in moe_last_cuda_error.
  * ------------------------------------------------------------------------- */
 #define MOE_NOALLOC_MAX_EXPERTS 256
 #define MOE_NOALLOC_SCRATCH_BYTES (256 + 256 * 256 * 4)

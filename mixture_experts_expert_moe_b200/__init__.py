@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_BF16, MOE_FP8_E4M3, MOE_F32 = 0, 1, 2
-MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN = 0x1, 0x2, 0x4
+MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN, MOE_DEV_DRAIN_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "combine"]
 
 EXPORTED = [

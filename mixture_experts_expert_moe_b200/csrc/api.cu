@@ -8,15 +8,21 @@
 #include "kernels.cuh"
 
 namespace {
-
 thread_local std::string g_last_cuda_error;
+}  // namespace
 
-moe_status_t cuda_fail(cudaError_t e, const char* where) {
+namespace moe {
+moe_status_t record_cuda_error(cudaError_t e, const char* where) {
   char buf[256];
   snprintf(buf, sizeof(buf), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
   g_last_cuda_error = buf;
   return MOE_ERR_CUDA;
 }
+}  // namespace moe
+
+namespace {
+
+inline moe_status_t cuda_fail(cudaError_t e, const char* where) { return moe::record_cuda_error(e, where); }
 
 #define MOE_CU(call)                                          \
   do {                                                        \

@@ -44,6 +44,9 @@ constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
 constexpr int kRing = 4;         // tile indices in flight from the producer to the other warps
+// after an abort, how long a CTA waits for its own copies and MMAs in flight
+// before it gives up (and reports MOE_DEV_DRAIN_TIMEOUT)
+constexpr long long kDrainTimeoutNs = 100000000LL;
 
 // Tile plan for the stand-alone FFN (moe_grouped_ffn), from the align & sort
 // outputs; layout in kernels.cuh, ordering in plan.cuh.
@@ -171,8 +174,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* t_empty = t_full + kRing;    // [kRing] every consumer has read it
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(t_empty + kRing);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  int* s_ring = s_abort + 1;    // [kRing]
-  int* s_start = s_ring + kRing + 2;
+  int* s_drain_fail = s_abort + 1;   // a drain after an abort ran out of time
+  int* s_ring = s_abort + 2;    // [kRing]
+  int* s_start = s_ring + kRing + 1;
   int* s_rows = s_start + E;
   int* s_groups = s_rows + E;
   int* s_perm = s_groups + E;
@@ -195,6 +199,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&t_empty[r], 9);   // the MMA thread and the 8 epilogue warps
     }
     *s_abort = 0;
+    *s_drain_fail = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
@@ -288,9 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < p.stages; ++s) {
           if (armed > s) {
             const uint32_t par = s < stage ? phase : phase ^ 1;
-            const unsigned long long t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[s], par) && (long long)(globaltimer_ns() - t0) < 100000000LL) {
-            }
+            if (!mbar_wait(&full[s], par, kDrainTimeoutNs)) *s_drain_fail = 1;
           }
         }
       }
@@ -359,9 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok && issued) {
         // wait for the MMAs in flight before TMEM is freed
         tc_commit(drain);
-        const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain, 0) && (long long)(globaltimer_ns() - t0) < 100000000LL) {
-        }
+        if (!mbar_wait(drain, 0, kDrainTimeoutNs)) *s_drain_fail = 1;
       }
     }
   } else {
@@ -465,6 +466,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) dev_flag(p.status, MOE_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && *s_drain_fail) dev_flag(p.status, MOE_DEV_DRAIN_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);

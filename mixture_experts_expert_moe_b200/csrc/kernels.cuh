@@ -4,6 +4,10 @@
 
 namespace moe {
 
+// Records "where: CUDA error text" for moe_last_cuda_error (this host thread)
+// and returns MOE_ERR_CUDA.
+moe_status_t record_cuda_error(cudaError_t e, const char* where);
+
 struct AlignParams {
   const int32_t* ids;
   int N;            // T*k flat slots

@@ -16,8 +16,12 @@
 // rejected with MOE_ERR_UNSUPPORTED before anything is launched.
 //
 // Set-up: the first call on each device (with that device current) looks up
-// the array's device address with cudaGetSymbolAddress and caches it; make
-// that first call before any stream capture.  Every later call on the device
+// the array's device address with cudaGetSymbolAddress and caches it per
+// device ordinal; make that first call before any stream capture.  The cached
+// address belongs to the device's primary context (the runtime API's
+// default): callers working in another context of the same device, or after
+// cudaDeviceReset on it, must not use this entry point (the address would
+// name memory of a context that is gone or not current).  Every later call on the device
 // reuses the same array, which keeps the previous call's contents: the
 // wait counter is cleared on the stream at the start of each call, and the
 // count matrix is fully rewritten before it is read.  Because all calls share
@@ -78,19 +82,24 @@ extern "C" MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, 
 
   int dev = 0, major = 0;
   const cudaError_t ge = cudaGetDevice(&dev);
-  if (ge == cudaErrorNoDevice || ge == cudaErrorInsufficientDriver) return MOE_ERR_DEVICE;
-  if (ge != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (ge == cudaErrorNoDevice || ge == cudaErrorInsufficientDriver) {
+    moe::record_cuda_error(ge, "cudaGetDevice");
+    return MOE_ERR_DEVICE;
+  }
+  if (ge != cudaSuccess) return moe::record_cuda_error(ge, "cudaGetDevice");
+  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return moe::record_cuda_error(e, "cudaDeviceGetAttribute");
   if (major != 10) return MOE_ERR_DEVICE;
 
   void* scratch = nullptr;
-  if (moe::scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  e = moe::scratch_address(&scratch);
+  if (e != cudaSuccess) return moe::record_cuda_error(e, "cudaGetSymbolAddress(align scratch)");
 
   // grid: one CTA per 4096 slots, at most one per SM (the kernel's co-residency rule)
   const int N = T * k;
   int err = 0;
   const int max_ctas = moe::align_max_ctas(E, &err);
-  if (err) return MOE_ERR_CUDA;
+  if (err) return moe::record_cuda_error((cudaError_t)err, "align occupancy");
   if (max_ctas < 1) return MOE_ERR_UNSUPPORTED;
   const int unit = 32 * 32;
   int grid = (int)(((long long)N + 4095) / 4096);
@@ -119,7 +128,9 @@ extern "C" MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, 
   p.expected = grid;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the shared wait counter must start at zero for every call
-  if (cudaMemsetAsync(p.barrier, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_align_sort(p, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+  e = cudaMemsetAsync(p.barrier, 0, sizeof(int), s);
+  if (e != cudaSuccess) return moe::record_cuda_error(e, "cudaMemsetAsync(align scratch counter)");
+  e = moe::launch_align_sort(p, grid, s);
+  if (e != cudaSuccess) return moe::record_cuda_error(e, "align & sort launch");
   return MOE_OK;
 }
