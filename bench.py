@@ -27,6 +27,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -37,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 from moe_inputs import ALIGN_CONFIG, CONFIGS, align_ids, make_layer  # noqa: E402
 from mixture_experts_expert_moe_b200.roofline import (  # noqa: E402
-    align_bytes, expert_weight_bytes, layer_bytes, moe_flops)
+    align_bytes, down_kernel_bytes, gateup_kernel_bytes, layer_bytes, moe_flops)
 
 METRIC = "MoE layer tokens/s & TFLOPS vs roofline (bf16/fp8); align&sort µs, GB/s"
 PRIMARY = CONFIGS["deepseek"]
@@ -77,7 +78,7 @@ class ClockSampler:
 
     def __init__(self, device):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"moe_bench_clocks_{os.getpid()}.csv")
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -85,7 +86,6 @@ class ClockSampler:
             self.gpu = str(device.index or 0)
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -106,14 +106,16 @@ class ClockSampler:
         self.f.close()
         rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) != 7:
-                    continue
-                try:
-                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
-                except ValueError:
-                    continue
+            lines = f.readlines()
+        os.remove(self.path)
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
         if not rows:
             return None
         smax = max(r[1] for r in rows)
@@ -128,8 +130,8 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0):
-    d = make_layer(cfg, device=dev)
+def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0, data=None):
+    d = make_layer(cfg, device=dev) if data is None else data
     if cfg.a8w8:
         layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype,
                            tile_tokens=tile_tokens, n_shared=cfg.n_shared, bias_mode=cfg.bias_mode)
@@ -250,40 +252,46 @@ def time_e2e(cfg, layer, d, steps, warmup):
 
 
 def gateup_bytes(cfg, touched):
-    eb = 1 if cfg.a8w8 else 2
-    pairs = slot_pairs(cfg)
-    w = touched * (2 * cfg.I * cfg.H * eb + (8 * cfg.I if cfg.a8w8 else 0))
-    return w + pairs * cfg.H * eb + pairs * cfg.I * 2
+    """Algorithmic bytes of one gate/up GEMM launch (touched gate+up weights
+    once, x once, routing)."""
+    return gateup_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8)
 
 
 def down_bytes(cfg, touched):
-    eb = 1 if cfg.a8w8 else 2
-    pairs = slot_pairs(cfg)
-    w = touched * (cfg.H * cfg.I * eb + (4 * cfg.H if cfg.a8w8 else 0))
-    return w + pairs * cfg.I * eb + pairs * cfg.H * 4     # + y, one fp32 row per slot
+    """Algorithmic bytes of one down GEMM launch (touched down weights once,
+    fp32 token outputs once, routing)."""
+    return down_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8)
 
 
-def traffic_for(kernel, workload):
-    """dram bytes per launch from the committed ncu summary table
-    (profiles/traffic.md), if it was taken on the current source of the kernel."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
-    if not os.path.exists(p):
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def traffic_for(kernel, workload, table=TRAFFIC_TABLE):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu traffic table, only while the kernel source still
+    has the hash recorded with the capture; None otherwise."""
+    if not os.path.exists(table):
         return None
-    for line in open(p):
-        cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) < 5 or cells[0] != kernel or cells[1] != workload:
+    with open(table) as f:
+        entries = json.load(f)["entries"]
+    for ent in entries:
+        if ent["kernel"] != kernel or ent["workload"] != workload:
             continue
-        src = os.path.join(ROOT, cells[3])
+        src = os.path.join(ROOT, ent["source"])
         if not os.path.exists(src):
             return None
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return int(cells[2]) if h == cells[4] else None
+        return int(ent["bytes_per_launch"]) if h == ent["sha256_16"] else None
     return None
 
 
-def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile_tokens=0):
-    d, layer = build_layer(m, cfg, dev, tile_tokens=tile_tokens)
-    touched, _ = touched_experts(layer, d)
+def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile_tokens=0, data=None):
+    """Time one workload (eager with stage events, then CUDA-graph replay) and
+    report it against its layer roofline and its dominant kernel's roofline.
+    ``data``: inputs from make_layer(cfg) to reuse (block-size sweeps)."""
+    d, layer = build_layer(m, cfg, dev, tile_tokens=tile_tokens, data=data)
+    touched, ids = touched_experts(layer, d)
+    load = torch.bincount(ids[:, :cfg.k].reshape(-1).long(), minlength=cfg.E)
     ms_eager, st = time_layer(m, cfg, layer, d, steps, warmup)
     ms_graph = time_graph(m, cfg, layer, d, steps, warmup)
     ms = ms_graph if ms_graph is not None else ms_eager
@@ -297,6 +305,7 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile
            "ms_per_step": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12, "touched_experts": touched,
            "layer_roofline_ms": t_roof, "layer_roofline_frac": t_roof / step_ms,
            "layer_bound": "tensor" if fl / (tf_peak * 1e12) > by / (pk["hbm_gbs"] * 1e9) else "hbm",
+           "max_tokens_per_expert": int(load.max().item()),
            "stages_ms": st, "launch": "cuda_graph" if ms_graph is not None else "eager",
            "eager_ms_per_step": ms_eager / steps}
     # dominant kernel
@@ -324,9 +333,27 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile
         ems, h2d, d2h = time_e2e(cfg, layer, d, max(10, steps // 2), 3)
         e2e = {"value": cfg.T * max(10, steps // 2) / (ems * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del layer, d
+    del layer
+    if data is None:
+        del d
     torch.cuda.empty_cache()
     return rep, e2e, ms
+
+
+def bm_sweep(m, cfg, steps, warmup, dev, pk, sizes=(32, 64, 128)):
+    """The layer at several block sizes (routing and values unchanged; the
+    padding and the GEMM token groups change), in bf16 and a8w8, each
+    precision's weights drawn once."""
+    out = []
+    for a8 in (False, True):
+        c = cfg.with_(a8w8=a8)
+        data = make_layer(c, device=dev)
+        for bm in sizes:
+            r, _, _ = layer_report(m, c.with_(bm=bm), steps, warmup, dev, pk, "a8w8" if a8 else "bf16", data=data)
+            out.append(r)
+        del data
+        torch.cuda.empty_cache()
+    return out
 
 
 def align_report(m, dev, pk, T, iters=100):
@@ -448,7 +475,11 @@ def run_ours(args):
 
     extra = {}
     if world == 1 and not args.quick:   # single-GPU reports (other ranks would idle in a barrier)
-        extra["a8w8"], _, _ = layer_report(m, cfg.with_(a8w8=True), 50, 5, dev, pk, "a8w8")
+        extra["deepseek_bm_sweep"] = bm_sweep(m, cfg, 30, 3, dev, pk)
+        extra["a8w8"] = next(r for r in extra["deepseek_bm_sweep"] if r["workload"].startswith("deepseek_a8w8")
+                             and r["workload"].endswith("bm=64"))
+        extra["deepseek_bias_4b"] = [layer_report(m, cfg.with_(bias=True, a8w8=a8), 30, 3, dev, pk,
+                                                  "a8w8" if a8 else "bf16")[0] for a8 in (False, True)]
         extra["mixtral"], _, _ = layer_report(m, CONFIGS["mixtral"], 20, 3, dev, pk, "bf16")
         extra["deepseek_shared"], _, _ = layer_report(m, CONFIGS["deepseek_shared"], 50, 5, dev, pk, "bf16")
         extra["decode_a8w8"] = []
@@ -460,6 +491,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(cfg)
+        if not args.quick:
+            extra["oracle_ops"] = oracle_op_times()
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -530,6 +563,80 @@ def _threads():
         return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         return os.cpu_count() or 1
+
+
+def cpu_model():
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def _timed(fn, min_s=0.5):
+    """Mean seconds per call of fn over enough calls to last min_s."""
+    fn()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            return dt / n
+
+
+def oracle_op_times(n_ffn_tokens=2):
+    """The oracle per step of the path, on the host cores, at one thread and at
+    every thread BLAS offers: gating of the DeepSeek-V3-shaped layer's 2048
+    tokens (top-8 of 256 logits), align & sort of the 16384-token Zipf
+    workload (top-8 of 256, block 64), both in full, and the expert FFN +
+    combine of a sample of that layer's tokens (bf16 weights)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        threadpool_limits = None
+    cfg = PRIMARY
+    logits = make_layer(cfg, device="cpu", weights=False)["logits"].numpy()
+    ids = align_ids(ALIGN_CONFIG["T"], ALIGN_CONFIG["E"], ALIGN_CONFIG["k"], seed=ALIGN_CONFIG["seed"],
+                    dist="zipf", zipf_s=ALIGN_CONFIG["zipf_s"])
+    x, lg, w13, w2 = _oracle_inputs(cfg, n_ffn_tokens, as_f32=False)
+    all_threads = _threads()
+    res = {"cpu_model": cpu_model(), "host_cpus": os.cpu_count(), "kind": "oracle", "levels": []}
+    for threads in sorted({1, all_threads}):
+        ctx = threadpool_limits(threads) if threadpool_limits else None
+        if ctx is not None:
+            ctx.__enter__()
+        try:
+            t_gate = _timed(lambda: oracle.topk_gate(logits, cfg.k))
+            t_align = _timed(lambda: oracle.align_sort(ids, ALIGN_CONFIG["E"], ALIGN_CONFIG["bm"]))
+            t0 = time.perf_counter()
+            oracle.moe_forward(x, lg, cfg.k, w13, w2)
+            t_ffn = time.perf_counter() - t0
+        finally:
+            if ctx is not None:
+                ctx.__exit__(None, None, None)
+        res["levels"].append({
+            "threads": threads,
+            "gate_ms": t_gate * 1e3, "gate_tokens_per_s": cfg.T / t_gate,
+            "align_sort_ms": t_align * 1e3,
+            "align_sort_slots_per_s": ALIGN_CONFIG["T"] * ALIGN_CONFIG["k"] / t_align,
+            "ffn_combine_s": t_ffn, "ffn_tokens_per_s": n_ffn_tokens / t_ffn})
+    res["sample"] = (f"gate: {cfg.T} x {cfg.E} logits, top-{cfg.k}; align & sort: {ALIGN_CONFIG['T']} tokens x "
+                     f"top-{ALIGN_CONFIG['k']} of {ALIGN_CONFIG['E']}, block {ALIGN_CONFIG['bm']}, in full; "
+                     f"FFN + combine: {n_ffn_tokens} seeded tokens of {workload_name(cfg, 'bf16')} "
+                     "(float64 numpy, bf16 weights converted per expert)")
+    return res
 
 
 def cpu_baseline(cfg, n_tokens=6):

@@ -39,3 +39,23 @@ def align_bytes(n_slots: int, num_post: int, block_size: int) -> int:
     """Algorithmic bytes of MoE Align & Sort: ids read once; sorted ids,
     per-block expert ids and the padded total written once."""
     return 4 * n_slots + 4 * num_post + 4 * (num_post // block_size) + 4
+
+
+def gateup_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool) -> int:
+    """Algorithmic bytes of the gate/up GEMM launch: the touched experts' gate
+    and up weights once (+ fp32 channel scales in a8w8), the tokens' x once
+    (at the operand precision) and the routing it reads (one sorted slot id
+    per pair).  The permuted copy of x, h and padding are not counted."""
+    eb = 1 if a8w8 else 2
+    w = touched * (2 * I * H * eb + (2 * I * 4 if a8w8 else 0))
+    return w + T * H * eb + pairs * 4
+
+
+def down_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool) -> int:
+    """Algorithmic bytes of the down GEMM launch: the touched experts' down
+    weights once (+ fp32 channel scales in a8w8), the fp32 token outputs
+    written once and the routing it reads (slot id and weight per pair).
+    The h operand and padding are not counted."""
+    eb = 1 if a8w8 else 2
+    w = touched * (H * I * eb + (H * 4 if a8w8 else 0))
+    return w + T * H * 4 + pairs * 8

@@ -47,3 +47,42 @@ class ExpertView:
         if self.codes:
             return x.view(__import__("torch").uint8).numpy()
         return x.float().numpy().astype(np.float64)
+
+
+def cover_sample(ids, n_hot=8, group_rows=(64, 128, 256)):
+    """Tokens whose outputs a full-size parity test compares, chosen from a
+    routing table ``ids`` [T, k] (the oracle's): the first and last token; a
+    greedy cover that reaches every expert in ``ids``; and, for the ``n_hot``
+    most loaded experts, the tokens of the last slot and of the first slot of
+    the last token group of each size in ``group_rows``.
+
+    Returns (sorted token indices, experts the sample reaches, experts touched).
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    T, k = ids.shape
+    chosen = {0, T - 1}
+    flat = ids.reshape(-1)
+    touched = np.unique(flat)
+    counts = np.bincount(flat, minlength=int(flat.max()) + 1)
+    for e in np.argsort(-counts, kind="stable")[:n_hot]:
+        slots = np.nonzero(flat == e)[0]          # ascending: the order inside the expert's segment
+        if slots.size == 0:
+            continue
+        chosen.add(int(slots[-1] // k))
+        for g in group_rows:
+            chosen.add(int(slots[((slots.size - 1) // g) * g] // k))
+    covered = set(flat[np.isin(np.arange(T * k) // k, list(chosen))].tolist())
+    member = np.zeros((T, counts.size), dtype=bool)
+    member[np.repeat(np.arange(T), k), flat] = True
+    missing = np.ones(counts.size, dtype=bool)
+    missing[list(covered)] = False
+    missing &= counts > 0
+    while missing.any():
+        gain = member[:, missing].sum(axis=1)
+        t = int(np.argmax(gain))
+        chosen.add(t)
+        missing &= ~member[t]
+        covered.update(np.nonzero(member[t])[0].tolist())
+    toks = np.array(sorted(chosen), dtype=np.int64)
+    reached = np.unique(ids[toks].reshape(-1)).size
+    return toks, int(reached), int(touched.size)

@@ -28,13 +28,21 @@ def test_kernels_per_step():
 def test_gateup_and_down_bytes_by_hand():
     cfg = MoEConfig("t", T=4, H=256, I=128, E=8, k=2, bm=16)
     touched = 3
-    # bf16: 3 experts x (2*128*256 weights x 2 B) + 8 pairs x 256 x 2 B (rows) + 8 pairs x 128 x 2 B (h)
-    assert bench.gateup_bytes(cfg, touched) == 3 * 2 * 128 * 256 * 2 + 8 * 256 * 2 + 8 * 128 * 2
-    # down: 3 x 256*128 x 2 + 8 x 128 x 2 (h) + 8 x 256 x 4 (fp32 y rows)
-    assert bench.down_bytes(cfg, touched) == 3 * 256 * 128 * 2 + 8 * 128 * 2 + 8 * 256 * 4
+    # bf16: 3 experts x (2*128*256 weights x 2 B) + x once (4 x 256 x 2 B) + 8 pairs x 4 B of slot ids
+    assert bench.gateup_bytes(cfg, touched) == 3 * 2 * 128 * 256 * 2 + 4 * 256 * 2 + 8 * 4
+    # down: 3 x 256*128 x 2 + fp32 token rows once (4 x 256 x 4) + 8 pairs x (slot id + weight)
+    assert bench.down_bytes(cfg, touched) == 3 * 256 * 128 * 2 + 4 * 256 * 4 + 8 * 8
     a8 = cfg.with_(a8w8=True)
-    # E4M3 weights + fp32 per-channel scales
-    assert bench.gateup_bytes(a8, touched) == 3 * (2 * 128 * 256 + 8 * 128) + 8 * 256 + 8 * 128 * 2
+    # E4M3 weights + fp32 per-channel scales; x at one byte per element
+    assert bench.gateup_bytes(a8, touched) == 3 * (2 * 128 * 256 + 2 * 128 * 4) + 4 * 256 + 8 * 4
+    assert bench.down_bytes(a8, touched) == 3 * (256 * 128 + 256 * 4) + 4 * 256 * 4 + 8 * 8
+
+
+def test_headline_kernel_bytes_are_the_weight_stream():
+    # DeepSeek-V3 gate/up: all 256 experts' gate+up weights dominate (15.03 GB of 15.06 GB)
+    cfg = CONFIGS["deepseek"]
+    b = bench.gateup_bytes(cfg, 256)
+    assert b == 256 * 2 * 2048 * 7168 * 2 + 2048 * 7168 * 2 + 2048 * 8 * 4
 
 
 def test_headline_workload_name():
@@ -43,9 +51,20 @@ def test_headline_workload_name():
     assert bench.workload_name(CONFIGS["deepseek_shared"], "bf16").endswith("+bias(selection only) +1 shared")
 
 
-def test_traffic_lookup_needs_matching_source():
+def test_traffic_lookup_needs_matching_source(tmp_path):
     # the committed table is keyed by the kernel source hash: a made-up workload has no entry
     assert bench.traffic_for("grouped_gemm_gateup", "no such workload") is None
+    import hashlib
+    import json
+    src = "mixture_experts_expert_moe_b200/roofline.py"
+    h = hashlib.sha256(open(os.path.join(bench.ROOT, src), "rb").read()).hexdigest()[:16]
+    t = tmp_path / "t.json"
+    ent = {"kernel": "k", "workload": "w", "bytes_per_launch": 123, "source": src, "sha256_16": h}
+    t.write_text(json.dumps({"entries": [ent]}))
+    assert bench.traffic_for("k", "w", table=str(t)) == 123
+    ent["sha256_16"] = "0" * 16          # the source changed since the capture
+    t.write_text(json.dumps({"entries": [ent]}))
+    assert bench.traffic_for("k", "w", table=str(t)) is None
 
 
 @pytest.mark.parametrize("world,units,steps,ms", [(1, 2048, 100, 400.0), (8, 2048, 50, 210.0)])

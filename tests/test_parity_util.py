@@ -1,0 +1,24 @@
+"""Host logic of the full-size parity sample (CPU)."""
+import numpy as np
+
+from parity_util import cover_sample
+
+
+def test_cover_sample_reaches_every_expert_and_the_hot_tails():
+    rng = np.random.default_rng(3)
+    T, E, k = 500, 40, 4
+    p = 1.0 / np.arange(1, E + 1)
+    ids = np.stack([rng.choice(E, size=k, replace=False, p=p / p.sum()) for _ in range(T)])
+    toks, reached, touched = cover_sample(ids, n_hot=3, group_rows=(16,))
+    assert reached == touched == np.unique(ids).size
+    assert toks[0] == 0 and toks[-1] == T - 1 and np.all(np.diff(toks) > 0)
+    flat = ids.reshape(-1)
+    for e in np.argsort(-np.bincount(flat, minlength=E), kind="stable")[:3]:
+        slots = np.nonzero(flat == e)[0]
+        assert slots[-1] // k in toks                               # last slot of a hot expert
+        assert slots[((slots.size - 1) // 16) * 16] // k in toks    # first slot of its last 16-row group
+
+
+def test_cover_sample_single_token():
+    toks, reached, touched = cover_sample(np.array([[3, 1, 2]]))
+    assert list(toks) == [0] and reached == touched == 3
