@@ -36,7 +36,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import ALIGN_CONFIG, CONFIGS, align_ids, make_layer  # noqa: E402
+from moe_inputs import ALIGN_CONFIG, CONFIGS, align_ids, make_layer, pack_e2m1  # noqa: E402
 from mixture_experts_expert_moe_b200.roofline import (  # noqa: E402
     align_bytes, down_kernel_bytes, gateup_kernel_bytes, layer_bytes, moe_flops)
 
@@ -132,7 +132,15 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0, data=None):
     d = make_layer(cfg, device=dev) if data is None else data
-    if cfg.a8w8:
+    if cfg.mx:
+        # model preparation: E2M1 codes packed two per byte, scales tiled for the MMA
+        pack = pack_e2m1 if cfg.mx == "mxfp4" else (lambda c: c)
+        w13, w2 = pack(d["w13_codes"]), pack(d["w2_codes"])
+        s13, s2 = m.mx_tile_scales(d["w13_sf"]), m.mx_tile_scales(d["w2_sf"])
+        layer = m.MoELayer(w13, w2, cfg.k, cfg.bm, out_dtype=out_dtype, tile_tokens=tile_tokens,
+                           n_shared=cfg.n_shared, bias_mode=cfg.bias_mode, mx=cfg.mx, w13_mx_scale=s13,
+                           w2_mx_scale=s2)
+    elif cfg.a8w8:
         layer = m.MoELayer(d["w13_q"], d["w2_q"], cfg.k, cfg.bm, d["w13_s"], d["w2_s"], out_dtype=out_dtype,
                            tile_tokens=tile_tokens, n_shared=cfg.n_shared, bias_mode=cfg.bias_mode)
     else:
@@ -173,7 +181,7 @@ def kernels_per_step(cfg, out_dtype):
     memset of the routing kernel's grid-wait counter is a runtime call, not a
     kernel of this library.)"""
     n = 5
-    if cfg.a8w8:
+    if cfg.a8w8 and not cfg.mx:
         n += 1 + (1 if slot_pairs(cfg) > 4096 else 0)
     return n
 
@@ -254,13 +262,13 @@ def time_e2e(cfg, layer, d, steps, warmup):
 def gateup_bytes(cfg, touched):
     """Algorithmic bytes of one gate/up GEMM launch (touched gate+up weights
     once, x once, routing)."""
-    return gateup_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8)
+    return gateup_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8, cfg.mx)
 
 
 def down_bytes(cfg, touched):
     """Algorithmic bytes of one down GEMM launch (touched down weights once,
     fp32 token outputs once, routing)."""
-    return down_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8)
+    return down_kernel_bytes(cfg.T, cfg.H, cfg.I, touched, slot_pairs(cfg), cfg.a8w8, cfg.mx)
 
 
 TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -298,8 +306,9 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile
     step_ms = ms / steps
     pairs = slot_pairs(cfg)
     fl = moe_flops(pairs, cfg.H, cfg.I)
-    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k + cfg.n_shared, touched, cfg.I, cfg.a8w8)
-    tf_peak = pk["bf16_tflops_sustained"] * (2.0 if cfg.a8w8 else 1.0)
+    by = layer_bytes(cfg.T, cfg.H, cfg.E, cfg.k + cfg.n_shared, touched, cfg.I, cfg.a8w8, mx=cfg.mx)
+    # E4M3 and MX (kind::mxf8f6f4, FP8 rate also with E2M1 weights): twice the bf16 tensor rate
+    tf_peak = pk["bf16_tflops_sustained"] * (2.0 if (cfg.a8w8 or cfg.mx) else 1.0)
     t_roof = max(fl / (tf_peak * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
     rep = {"workload": workload_name(cfg, dtype_name), "tokens_per_s": cfg.T / (step_ms * 1e-3),
            "ms_per_step": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12, "touched_experts": touched,
@@ -486,6 +495,13 @@ def run_ours(args):
         for T in (1, 16, 64, 256):
             r, _, _ = layer_report(m, CONFIGS["decode"].with_(T=T), 100, 5, dev, pk, "a8w8")
             extra["decode_a8w8"].append(r)
+        extra["decode_mx"] = []
+        for fmt in ("mxfp4", "mxfp8"):
+            for T in (1, 16, 64, 256):
+                c = CONFIGS["decode"].with_(T=T, a8w8=False, mx=fmt)
+                extra["decode_mx"].append(layer_report(m, c, 100, 5, dev, pk, fmt)[0])
+        extra["deepseek_mx"] = [layer_report(m, cfg.with_(mx=fmt), 30, 3, dev, pk, fmt)[0]
+                                for fmt in ("mxfp4", "mxfp8")]
         extra["align_sort"] = align_report(m, dev, pk, ALIGN_CONFIG["T"])
         extra["align_sort_large"] = align_report(m, dev, pk, 1 << 22, iters=20)
     cpu = None
@@ -692,7 +708,7 @@ def run_only(args):
         return
     if len(parts) > 2 and f"{parts[0]}_{parts[1]}" in CONFIGS:     # e.g. deepseek_shared
         parts = [f"{parts[0]}_{parts[1]}"] + parts[2:]
-    cfg = CONFIGS[parts[0]].with_(a8w8=parts[1] == "a8w8")
+    cfg = CONFIGS[parts[0]].with_(a8w8=parts[1] == "a8w8", mx=parts[1] if parts[1].startswith("mx") else "")
     tile = 0
     for p in parts[2:]:
         if p.startswith("bm"):
@@ -718,7 +734,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--only", default=None,
-                    help="time one workload and print its report: <config>_<bf16|a8w8>[_bm<N>][_T<N>][_E<N>][_tn<N>] "
+                    help="time one workload and print its report: <config>_<bf16|a8w8|mxfp8|mxfp4>"
+                         "[_bm<N>][_T<N>][_E<N>][_tn<N>] "
                          "(configs: tiny, p5, deepseek, deepseek_shared, mixtral, decode) or align_<T>")
     args = ap.parse_args()
     if args.only:

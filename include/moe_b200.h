@@ -62,7 +62,10 @@ typedef enum {
                                 driver at all, or another architecture      */
 } moe_status_t;
 
-typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2 } moe_dtype_t;
+/* MOE_MXFP8 / MOE_MXFP4: MX block-scaled weights (OCP Microscaling: one E8M0
+ * scale per 32 consecutive elements along K; E4M3 or E2M1 elements); the
+ * activations are then MXFP8 too (see moe_grouped_ffn). */
+typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2, MOE_MXFP8 = 3, MOE_MXFP4 = 4 } moe_dtype_t;
 
 /* Device-side status bits (OR-ed into *dev_status). */
 #define MOE_DEV_BAD_EXPERT_ID 0x1  /* an expert id outside [0, E): slot skipped */
@@ -80,8 +83,10 @@ MOE_API const char* moe_status_string(int status);
 MOE_API const char* moe_last_cuda_error(void);
 /* ABI version (major*100 + minor); equals MOE_ABI_VERSION of the header the
  * library was built with.  Major 2: moe_topk_gate takes bias_mode and
- * n_shared, moe_forward_args ends with n_shared and bias_mode. */
-#define MOE_ABI_VERSION 200
+ * n_shared, moe_forward_args ends with n_shared and bias_mode.  Major 3:
+ * moe_ffn_args and moe_forward_args end with the MX weight scales; MX weight
+ * types; moe_mx_tile_scales, moe_mx_quantize_rows. */
+#define MOE_ABI_VERSION 300
 MOE_API int moe_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -185,6 +190,13 @@ MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, int T, int 
  *          g = (Wg_q[e] q_x) * s_x * w13_scale[e], u likewise,
  *          h = bf16(silu(g) * u), (q_h, s_h) = per-row requantisation,
  *          y_s = (Wd_q[e] q_h) * s_h * w2_scale[e]
+ *   MX (MOE_MXFP8 / MOE_MXFP4 weights; GC-MoE abstract: block-scaled MMAs
+ *   with FP4 weights on Blackwell):
+ *          x_t is MXFP8-quantised (per 32 elements along H: X = 2^(floor(log2
+ *          amax) - 8), E4M3 codes of x / X), g and u are the block sums
+ *          sum_b X_x[b] X_w[n,b] (q_x[b] . q_w[n,b]) accumulated in fp32,
+ *          h = bf16(silu(g) * u) is MXFP8-quantised along I in the gate/up
+ *          GEMM's epilogue (no separate requantisation), y_s likewise.
  * ------------------------------------------------------------------------- */
 typedef struct {
   int T, H, I, E, k, block_size;
@@ -199,11 +211,19 @@ typedef struct {
   const int32_t* expert_ids;  /* [NB] from moe_align_sort                        */
   const int32_t* num_post;    /* [1]  from moe_align_sort                        */
   int tile_tokens;            /* tokens per GEMM tile: 0 = automatic, else one
-                                 of 16, 32, 64, 128, 256                          */
+                                 of 16, 32, 64, 128, 256 (MX: at most 128)        */
+  /* MX weights only (else NULL): E8M0 scale codes in the tiled layout of
+   * moe_mx_tile_scales, from [E * 2I, H/32] and [E * H, I/32].  With MX
+   * weights w13 / w2 hold E4M3 codes [E, 2I, H] / [E, H, I] (MOE_MXFP8) or E2M1
+   * codes packed two per byte, element 2j in the low nibble, [E, 2I, H/2] /
+   * [E, H, I/2] (MOE_MXFP4; 32-byte aligned). */
+  const uint8_t* w13_mx_scale;
+  const uint8_t* w2_mx_scale;
 } moe_ffn_args;
 
 /* Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32,
- * 1 <= block_size <= 1024; device pointers 16-byte aligned. */
+ * 1 <= block_size <= 1024; device pointers 16-byte aligned (MXFP4 weights:
+ * 32-byte).  Missing scales for the weight type: MOE_ERR_INVALID_ARG. */
 MOE_API moe_status_t moe_ffn_workspace(const moe_ffn_args* args, size_t* ws_bytes);
 /*   y  f32 [T*k, H]  out: per-slot expert output y_s (rows of slots that were
  *                    skipped are not written) */
@@ -260,6 +280,8 @@ typedef struct {
                                  `stream` (for per-stage timing)           */
   int n_shared;               /* shared experts after the E routed ones (0..) */
   int bias_mode;              /* MOE_BIAS_LOGITS or MOE_BIAS_SELECT        */
+  const uint8_t* w13_mx_scale;  /* MX weights only: as in moe_ffn_args      */
+  const uint8_t* w2_mx_scale;
 } moe_forward_args;
 
 /* Stages of moe_forward, in launch order (stage_events indices). */
@@ -277,6 +299,31 @@ typedef struct {
 MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);
 MOE_API moe_status_t moe_forward(const moe_forward_args* args, void* ws, size_t ws_bytes,
                          int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_mx_tile_scales -- lay out MX weight scales for the block-scaled GEMM.
+ * Model preparation, done once per weight tensor (GC-MoE abstract: block-
+ * scaled MMAs; the scale layout is the one the tensor cores' scale-factor
+ * copies read, 128 rows x 4 K-blocks per 512-byte chunk).
+ *   sf   u8 [rows, K/32]  E8M0 scale codes, one per 32 elements of a row
+ *   out  u8 [rows * K/32] chunk (rt, w) = rows 128*rt.. x K-blocks 4w..4w+3
+ *        holds at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + b the scale of
+ *        row 128*rt + r, K-block 4w + b; chunks ordered rt-major.
+ * Limits: rows % 128 == 0, K % 128 == 0, 16-byte aligned pointers.
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_mx_tile_scales(const uint8_t* sf, long long rows, int K, uint8_t* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_mx_quantize_rows -- MXFP8 quantisation of bf16 rows (the activation
+ * quantiser of the MX path, also usable on its own).
+ *   x       bf16 [R, C];  codes u8 [R, C] out: E4M3 codes of x / X
+ *   scales  u8 [R, C/32] out: E8M0 code 127 + floor(log2 amax) - 8 of every
+ *           32-element block (clamped to >= 0; 127 for an all-zero block)
+ * Rounding: nearest even, saturating to +-448.  Limits: C % 32 == 0, R >= 0,
+ * 16-byte aligned x and codes.
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_mx_quantize_rows(const void* x, int R, int C, uint8_t* codes, uint8_t* scales,
+                                          void* stream);
 
 /* ---------------------------------------------------------------------------
  * Diagnostics.

@@ -16,7 +16,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
-MOE_BF16, MOE_FP8_E4M3, MOE_F32 = 0, 1, 2
+MOE_BF16, MOE_FP8_E4M3, MOE_F32, MOE_MXFP8, MOE_MXFP4 = 0, 1, 2, 3, 4
+_MX_TYPES = {"mxfp8": MOE_MXFP8, "mxfp4": MOE_MXFP4}
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN, MOE_DEV_DRAIN_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "combine"]
 
@@ -24,7 +25,7 @@ EXPORTED = [
     "moe_status_string", "moe_last_cuda_error", "moe_version", "moe_topk_gate",
     "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
     "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
-    "moe_align_sort_noalloc", "moe_test_quant_division",
+    "moe_align_sort_noalloc", "moe_test_quant_division", "moe_mx_tile_scales", "moe_mx_quantize_rows",
 ]
 
 _vp = ctypes.c_void_p
@@ -35,7 +36,7 @@ class FfnArgs(ctypes.Structure):
     _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i),
                 ("wdtype", _i), ("x", _vp), ("w13", _vp), ("w13_scale", _vp), ("w2", _vp),
                 ("w2_scale", _vp), ("sorted_ids", _vp), ("expert_ids", _vp), ("num_post", _vp),
-                ("tile_tokens", _i)]
+                ("tile_tokens", _i), ("w13_mx_scale", _vp), ("w2_mx_scale", _vp)]
 
 
 class ForwardArgs(ctypes.Structure):
@@ -43,11 +44,11 @@ class ForwardArgs(ctypes.Structure):
                 ("wdtype", _i), ("out_dtype", _i), ("x", _vp), ("logits", _vp), ("bias", _vp),
                 ("w13", _vp), ("w13_scale", _vp), ("w2", _vp), ("w2_scale", _vp), ("out", _vp),
                 ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i), ("stage_events", _vp),
-                ("n_shared", _i), ("bias_mode", _i)]
+                ("n_shared", _i), ("bias_mode", _i), ("w13_mx_scale", _vp), ("w2_mx_scale", _vp)]
 
 
 MOE_BIAS_LOGITS, MOE_BIAS_SELECT = 0, 1
-ABI_VERSION = 200   # MOE_ABI_VERSION of include/moe_b200.h
+ABI_VERSION = 300   # MOE_ABI_VERSION of include/moe_b200.h
 _BIAS_MODES = {"logits": MOE_BIAS_LOGITS, "select": MOE_BIAS_SELECT}
 
 
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_test_wait_timeout": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
             "moe_align_sort_noalloc": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
             "moe_test_quant_division": (_i, [_vp, _vp]),
+            "moe_mx_tile_scales": (_i, [_vp, ctypes.c_longlong, _i, _vp, _vp]),
+            "moe_mx_quantize_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -117,12 +120,21 @@ def _dev_status(dev_status, device):
     return _ptr(dev_status)
 
 
-def _wdtype(w):
+def _wdtype(w, mx=None):
+    if mx is not None:
+        if w.dtype != torch.uint8:
+            raise TypeError("MX weights are uint8 codes (E4M3, or E2M1 packed two per byte)")
+        return _MX_TYPES[mx]
     if w.dtype == torch.bfloat16:
         return MOE_BF16
     if w.dtype in (torch.float8_e4m3fn, torch.uint8):
         return MOE_FP8_E4M3
     raise TypeError(f"unsupported weight dtype {w.dtype}")
+
+
+def _inner_k(w, mx):
+    """Elements along K of a weight tensor (E2M1 codes are packed two per byte)."""
+    return w.shape[-1] * (2 if mx == "mxfp4" else 1)
 
 
 # ---------------------------------------------------------------------------
@@ -174,26 +186,30 @@ def align_sort(topk_ids: torch.Tensor, E: int, block_size: int, dev_status=None,
 
 
 def _ffn_args(x, w13, w2, sorted_ids, expert_ids, num_post, T, k, E, block_size, w13_scale, w2_scale,
-              tile_tokens):
+              tile_tokens, mx=None, w13_mx_scale=None, w2_mx_scale=None):
     H = x.shape[1]
     I = w13.shape[1] // 2
-    a = FfnArgs(T=T, H=H, I=I, E=E, k=k, block_size=block_size, wdtype=_wdtype(w13),
+    a = FfnArgs(T=T, H=H, I=I, E=E, k=k, block_size=block_size, wdtype=_wdtype(w13, mx),
                 x=x.data_ptr(), w13=w13.data_ptr(), w2=w2.data_ptr(),
                 w13_scale=None if w13_scale is None else w13_scale.data_ptr(),
                 w2_scale=None if w2_scale is None else w2_scale.data_ptr(),
                 sorted_ids=sorted_ids.data_ptr(), expert_ids=expert_ids.data_ptr(),
-                num_post=num_post.data_ptr(), tile_tokens=tile_tokens)
+                num_post=num_post.data_ptr(), tile_tokens=tile_tokens,
+                w13_mx_scale=None if w13_mx_scale is None else w13_mx_scale.data_ptr(),
+                w2_mx_scale=None if w2_mx_scale is None else w2_mx_scale.data_ptr())
     return a
 
 
 def grouped_ffn(x, w13, w2, sorted_ids, expert_ids, num_post, k, block_size, w13_scale=None, w2_scale=None,
-                tile_tokens=0, dev_status=None, y=None, ws=None):
-    """Per-slot expert FFN output y f32 [T*k, H] over align&sort's outputs."""
+                tile_tokens=0, dev_status=None, y=None, ws=None, mx=None, w13_mx_scale=None, w2_mx_scale=None):
+    """Per-slot expert FFN output y f32 [T*k, H] over align&sort's outputs.
+    ``mx`` ("mxfp8" / "mxfp4"): MX weights (uint8 codes) with tiled E8M0
+    scales ``w13_mx_scale`` / ``w2_mx_scale`` from ``mx_tile_scales``."""
     lib = load_library()
     T, H = x.shape
     E = w13.shape[0]
     a = _ffn_args(x, w13, w2, sorted_ids, expert_ids, num_post, T, k, E, block_size, w13_scale, w2_scale,
-                  tile_tokens)
+                  tile_tokens, mx, w13_mx_scale, w2_mx_scale)
     nbytes = ctypes.c_size_t()
     _check(lib.moe_ffn_workspace(ctypes.byref(a), ctypes.byref(nbytes)), "moe_ffn_workspace")
     if ws is None:
@@ -229,12 +245,14 @@ class MoELayer:
     """
 
     def __init__(self, w13, w2, k, block_size, w13_scale=None, w2_scale=None, out_dtype=torch.bfloat16,
-                 tile_tokens=0, n_shared=0, bias_mode="logits"):
+                 tile_tokens=0, n_shared=0, bias_mode="logits", mx=None, w13_mx_scale=None, w2_mx_scale=None):
         self.w13, self.w2, self.k, self.block_size = w13, w2, k, block_size
         self.w13_scale, self.w2_scale = w13_scale, w2_scale
+        self.mx, self.w13_mx_scale, self.w2_mx_scale = mx, w13_mx_scale, w2_mx_scale
         self.out_dtype, self.tile_tokens = out_dtype, tile_tokens
         self.n_shared, self.bias_mode = n_shared, _BIAS_MODES[bias_mode]
-        EW, twoI, self.H = w13.shape
+        EW, twoI, _ = w13.shape
+        self.H = _inner_k(w13, mx)
         self.E = EW - n_shared
         self.I = twoI // 2
         self._ws = None
@@ -243,19 +261,21 @@ class MoELayer:
         T = x.shape[0]
         return ForwardArgs(
             T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
-            wdtype=_wdtype(self.w13), out_dtype=MOE_BF16 if out.dtype == torch.bfloat16 else MOE_F32,
+            wdtype=_wdtype(self.w13, self.mx), out_dtype=MOE_BF16 if out.dtype == torch.bfloat16 else MOE_F32,
             x=x.data_ptr(), logits=logits.data_ptr(), bias=None if bias is None else bias.data_ptr(),
             w13=self.w13.data_ptr(), w13_scale=None if self.w13_scale is None else self.w13_scale.data_ptr(),
             w2=self.w2.data_ptr(), w2_scale=None if self.w2_scale is None else self.w2_scale.data_ptr(),
             out=out.data_ptr(), topk_ids=None if ids is None else ids.data_ptr(),
             topk_w=None if w is None else w.data_ptr(), tile_tokens=self.tile_tokens,
             stage_events=None if events is None else ctypes.cast(events, ctypes.c_void_p),
-            n_shared=self.n_shared, bias_mode=self.bias_mode)
+            n_shared=self.n_shared, bias_mode=self.bias_mode,
+            w13_mx_scale=None if self.w13_mx_scale is None else self.w13_mx_scale.data_ptr(),
+            w2_mx_scale=None if self.w2_mx_scale is None else self.w2_mx_scale.data_ptr())
 
     def workspace_bytes(self, T):
         lib = load_library()
         a = ForwardArgs(T=T, H=self.H, I=self.I, E=self.E, k=self.k, block_size=self.block_size,
-                        wdtype=_wdtype(self.w13),
+                        wdtype=_wdtype(self.w13, self.mx),
                         out_dtype=MOE_BF16 if self.out_dtype == torch.bfloat16 else MOE_F32,
                         tile_tokens=self.tile_tokens, n_shared=self.n_shared, bias_mode=self.bias_mode)
         n = ctypes.c_size_t()
@@ -284,6 +304,32 @@ class MoELayer:
         _check(lib.moe_forward(ctypes.byref(a), _ptr(self._ws), self._ws.numel(),
                                _dev_status(dev_status, x.device), _stream(x.device)), "moe_forward")
         return out
+
+
+def mx_tile_scales(sf: torch.Tensor) -> torch.Tensor:
+    """Per-row E8M0 weight scales ``sf`` uint8 [..., rows, K/32] (any leading
+    dims folded into rows; rows % 128 == 0, K % 128 == 0) rearranged into the
+    tiled layout the MX grouped GEMM reads (model preparation, done once)."""
+    lib = load_library()
+    assert sf.is_cuda and sf.dtype == torch.uint8 and sf.is_contiguous()
+    K = sf.shape[-1] * 32
+    rows = sf.numel() // sf.shape[-1]
+    out = torch.empty_like(sf)
+    _check(lib.moe_mx_tile_scales(_ptr(sf), rows, K, _ptr(out), _stream(sf.device)), "moe_mx_tile_scales")
+    return out
+
+
+def mx_quantize_rows(x: torch.Tensor):
+    """MXFP8 quantisation of bf16 rows x [R, C]: (E4M3 codes uint8 [R, C],
+    E8M0 scale codes uint8 [R, C/32])."""
+    lib = load_library()
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    R, C = x.shape
+    codes = torch.empty(R, C, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(R, C // 32, dtype=torch.uint8, device=x.device)
+    _check(lib.moe_mx_quantize_rows(_ptr(x), R, C, _ptr(codes), _ptr(scales), _stream(x.device)),
+           "moe_mx_quantize_rows")
+    return codes, scales
 
 
 def capture_graph(layer, x, logits, bias=None, out=None):

@@ -125,6 +125,7 @@ moe_status_t run_align(const int32_t* ids, int T, int k, int E, int bm, int32_t*
 // ---------------------------------------------------------------------------
 struct FfnShape {
   int T, H, I, E, k, bm, fp8, tn;
+  int mx, fp4;          // MX block-scaled operands; E2M1 weights
   long long P, NB, N;
   long long rows_max;   // bound on num_post: at most min(E, N) experts pad, each by < bm rows
 };
@@ -134,20 +135,27 @@ int pick_tn(const FfnShape& s, int hint) {
   const double avg = (double)s.N / s.E;  // slots per expert
   long long need = (long long)((avg * 1.25 + s.bm - 1) / s.bm) * s.bm;
   if (need < s.bm) need = s.bm;
+  // MX tiles stage every stage's activation scales of two token tiles in
+  // shared memory, which leaves room for at most 128 tokens per tile
+  const int cap = s.mx ? 128 : 256;
   int tn = 16;
-  while (tn < need && tn < 256) tn <<= 1;
+  while (tn < need && tn < cap) tn <<= 1;
   return tn;
 }
 
 moe_status_t ffn_shape(int T, int H, int I, int E, int k, int bm, int wdtype, int hint, FfnShape* s) {
   if (!align_args_ok(T, k, E, bm) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
   if (k > 32 || k > E) return MOE_ERR_INVALID_ARG;
-  if (wdtype != MOE_BF16 && wdtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (wdtype != MOE_BF16 && wdtype != MOE_FP8_E4M3 && wdtype != MOE_MXFP8 && wdtype != MOE_MXFP4)
+    return MOE_ERR_INVALID_ARG;
   if (hint != 0 && hint != 16 && hint != 32 && hint != 64 && hint != 128 && hint != 256)
     return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128) return MOE_ERR_UNSUPPORTED;
   s->T = T; s->H = H; s->I = I; s->E = E; s->k = k; s->bm = bm;
   s->fp8 = wdtype == MOE_FP8_E4M3;
+  s->mx = wdtype == MOE_MXFP8 || wdtype == MOE_MXFP4;
+  s->fp4 = wdtype == MOE_MXFP4;
+  if (s->mx && hint > 128) return MOE_ERR_UNSUPPORTED;
   s->N = (long long)T * k;
   s->P = s->N + (long long)E * (bm - 1);
   s->NB = (s->P + bm - 1) / bm;
@@ -165,17 +173,21 @@ struct FfnWs {
   size_t plan, xq, sx, A, sA, h, hq, sH, total;
 };
 
+// Workspace: the tile plan; the sorted activations A (bf16, E4M3 + a scale
+// per row, or MX: E4M3 + E8M0 per 32 elements); h (bf16), and in FP8 / MX
+// its quantised copy hq with its scales (MX: h is quantised by the gate/up
+// epilogue, so only hq exists).
 FfnWs ffn_ws_layout(const FfnShape& s) {
   Carver c;
   FfnWs w;
   w.plan = c.take((size_t)moe::plan_ints(s.E) * 4);
   w.xq = c.take(s.fp8 ? (size_t)s.T * s.H : 0);
   w.sx = c.take(s.fp8 ? (size_t)s.T * 4 : 0);
-  w.A = c.take((size_t)s.P * s.H * (s.fp8 ? 1 : 2));
-  w.sA = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
-  w.h = c.take((size_t)s.P * s.I * 2);
-  w.hq = c.take(s.fp8 ? (size_t)s.P * s.I : 0);
-  w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : 0);
+  w.A = c.take((size_t)s.P * s.H * (s.fp8 || s.mx ? 1 : 2));
+  w.sA = c.take(s.fp8 ? (size_t)s.P * 4 : s.mx ? (size_t)s.P * (s.H / 32) : 0);
+  w.h = c.take(s.mx ? 0 : (size_t)s.P * s.I * 2);
+  w.hq = c.take(s.fp8 || s.mx ? (size_t)s.P * s.I : 0);
+  w.sH = c.take(s.fp8 ? (size_t)s.P * 4 : s.mx ? (size_t)s.P * (s.I / 32) : 0);
   w.total = c.off;
   return w;
 }
@@ -189,10 +201,24 @@ moe_status_t gemm_fail(int r, const char* what) {
 }
 
 // Runs plan -> gather(+quant) -> gate/up GEMM -> (requant) -> down GEMM.
-moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const float* w13s, const void* w2,
-                     const float* w2s, const int32_t* sorted, const int32_t* expert_ids, const int32_t* num_post,
-                     float* y, uint8_t* ws, int32_t* status, cudaStream_t stream, void** ev = nullptr,
-                     bool plan_ready = false, float* comb_out = nullptr, const float* comb_w = nullptr) {
+// Weight operands of one FFN call.
+struct FfnWeights {
+  const void* w13;
+  const float* w13s;          // FP8: per-channel scales
+  const void* w2;
+  const float* w2s;
+  const uint8_t* w13_mx;      // MX: tiled E8M0 scales
+  const uint8_t* w2_mx;
+};
+
+moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, const int32_t* sorted,
+                     const int32_t* expert_ids, const int32_t* num_post, float* y, uint8_t* ws, int32_t* status,
+                     cudaStream_t stream, void** ev = nullptr, bool plan_ready = false, float* comb_out = nullptr,
+                     const float* comb_w = nullptr) {
+  const void* w13 = W.w13;
+  const void* w2 = W.w2;
+  const float* w13s = W.w13s;
+  const float* w2s = W.w2s;
   const FfnWs L = ffn_ws_layout(s);
   int32_t* plan = reinterpret_cast<int32_t*>(ws + L.plan);
   void* A = ws + L.A;
@@ -209,7 +235,11 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
     MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status,
                             stream));
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
-  if (s.fp8 && N <= kFusedQuantSlots) {
+  if (s.mx) {
+    // every sorted row MX-quantises its token (codes + a scale per 32 elements)
+    MOE_CU(moe::launch_mx_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, reinterpret_cast<uint8_t*>(sA),
+                                     stream));
+  } else if (s.fp8 && N <= kFusedQuantSlots) {
     // few slots: each sorted row quantises its token directly (one launch)
     MOE_CU(moe::launch_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, sA, status, stream));
   } else if (s.fp8) {
@@ -228,6 +258,11 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.x_rows = s.P;
   g1.p.gateup = 1;
   g1.p.fp8 = s.fp8;
+  g1.p.mx = s.mx;
+  g1.p.w_fp4 = s.fp4;
+  g1.p.w_sf = W.w13_mx;
+  g1.p.x_sf = reinterpret_cast<const uint8_t*>(sA);
+  g1.p.h_sf = reinterpret_cast<uint8_t*>(sH);
   g1.p.K = s.H;
   g1.p.n_out = s.I;
   g1.p.tn = s.tn;
@@ -238,7 +273,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   g1.p.sorted = sorted;
   g1.p.a_scale = sA;
   g1.p.w_scale = w13s;
-  g1.p.out = h;
+  g1.p.out = s.mx ? hq : h;   // MX: the epilogue writes the MXFP8 codes of h (+ their scales)
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
   g1.p.tile_counter = plan + moe::plan_counter(s.E, true);
@@ -252,10 +287,14 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   moe::GemmLaunch g2 = {};
   g2.w = w2;
   g2.w_rows = (long long)s.E * s.H;
-  g2.x = s.fp8 ? hq : h;
+  g2.x = s.fp8 || s.mx ? hq : h;
   g2.x_rows = s.P;
   g2.p.gateup = 0;
   g2.p.fp8 = s.fp8;
+  g2.p.mx = s.mx;
+  g2.p.w_fp4 = s.fp4;
+  g2.p.w_sf = W.w2_mx;
+  g2.p.x_sf = reinterpret_cast<const uint8_t*>(sH);
   g2.p.K = s.I;
   g2.p.n_out = s.H;
   g2.p.tn = s.tn;
@@ -276,6 +315,16 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const void* w13, const fl
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
   return MOE_OK;
+}
+
+// The weight pointers and scales a weight type needs, aligned for TMA.
+bool weights_ok(const FfnShape& s, const void* w13, const float* w13s, const void* w2, const float* w2s,
+                       const uint8_t* w13_mx, const uint8_t* w2_mx) {
+  if (!w13 || !w2) return false;
+  if (s.fp8 && (!w13s || !w2s)) return false;
+  if (s.mx && (!w13_mx || !w2_mx || !aligned16(w13_mx) || !aligned16(w2_mx))) return false;
+  const uintptr_t a = s.fp4 ? 31 : 15;   // packed 4-bit tensor maps need 32-byte aligned bases
+  return ((reinterpret_cast<uintptr_t>(w13) | reinterpret_cast<uintptr_t>(w2)) & a) == 0;
 }
 
 // Gate + align&sort + tile plan in one launch (moe_forward).
@@ -413,14 +462,15 @@ moe_status_t moe_grouped_ffn(const moe_ffn_args* a, float* y, void* ws, size_t w
   if (s.N == 0) return MOE_OK;
   if (!a->x || !a->w13 || !a->w2 || !a->sorted_ids || !a->expert_ids || !a->num_post || !y || !ws)
     return MOE_ERR_INVALID_ARG;
-  if (s.fp8 && (!a->w13_scale || !a->w2_scale)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(a->x) || !aligned16(a->w13) || !aligned16(a->w2) || !aligned16(y) || !aligned16(ws))
+  if (!weights_ok(s, a->w13, a->w13_scale, a->w2, a->w2_scale, a->w13_mx_scale, a->w2_mx_scale))
     return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->x) || !aligned16(y) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < ffn_ws_layout(s).total) return MOE_ERR_WORKSPACE;
   st = check_device();
   if (st) return st;
-  return run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, a->sorted_ids, a->expert_ids, a->num_post,
-                 y, static_cast<uint8_t*>(ws), dev_status, (cudaStream_t)stream);
+  const FfnWeights W = {a->w13, a->w13_scale, a->w2, a->w2_scale, a->w13_mx_scale, a->w2_mx_scale};
+  return run_ffn(s, a->x, W, a->sorted_ids, a->expert_ids, a->num_post, y, static_cast<uint8_t*>(ws), dev_status,
+                 (cudaStream_t)stream);
 }
 
 moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int H, void* out, int out_dtype,
@@ -496,10 +546,10 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   moe_status_t st = forward_shape(a, &s);
   if (st) return st;
   if (s.T == 0) return MOE_OK;
-  if (!a->x || !a->logits || !a->w13 || !a->w2 || !a->out || !ws) return MOE_ERR_INVALID_ARG;
-  if (s.fp8 && (!a->w13_scale || !a->w2_scale)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(a->x) || !aligned16(a->w13) || !aligned16(a->w2) || !aligned16(a->out) || !aligned16(ws))
+  if (!a->x || !a->logits || !a->out || !ws) return MOE_ERR_INVALID_ARG;
+  if (!weights_ok(s, a->w13, a->w13_scale, a->w2, a->w2_scale, a->w13_mx_scale, a->w2_mx_scale))
     return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->x) || !aligned16(a->out) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   const FwdWs L = fwd_ws_layout(s, a->out_dtype);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   st = check_device();
@@ -528,8 +578,8 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
   // fused: the down GEMM adds w * y of every slot into its token's fp32 row;
   // otherwise it writes y per slot and the combine kernel sums them
-  st = run_ffn(s, a->x, a->w13, a->w13_scale, a->w2, a->w2_scale, sorted, eids, npost, y, ffn_ws, dev_status,
-               cs, ev, /*plan_ready=*/true, out32, tw);
+  const FfnWeights W = {a->w13, a->w13_scale, a->w2, a->w2_scale, a->w13_mx_scale, a->w2_mx_scale};
+  st = run_ffn(s, a->x, W, sorted, eids, npost, y, ffn_ws, dev_status, cs, ev, /*plan_ready=*/true, out32, tw);
   if (st) return st;
   if (fused) {
     if (out_bf16) MOE_CU(moe::launch_cast_bf16(out32, (long long)s.T * s.H, a->out, cs));
@@ -537,6 +587,26 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
     MOE_CU(moe::launch_combine(y, tw, s.T, s.k, s.H, a->out, out_bf16, cs));
   }
   MOE_CU(record(ev, MOE_STAGE_COMBINE + 1, cs));
+  return MOE_OK;
+}
+
+moe_status_t moe_mx_tile_scales(const uint8_t* sf, long long rows, int K, uint8_t* out, void* stream) {
+  if (rows < 0 || K < 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+  if (rows == 0 || K == 0) return MOE_OK;
+  if (!sf || !out || !aligned16(sf) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_mx_tile_scales(sf, rows, K, out, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status_t moe_mx_quantize_rows(const void* x, int R, int C, uint8_t* codes, uint8_t* scales, void* stream) {
+  if (R < 0 || C < 0 || C % 32) return MOE_ERR_INVALID_ARG;
+  if (R == 0 || C == 0) return MOE_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_mx_quant_rows(x, nullptr, 0, 1, nullptr, R, C, codes, scales, (cudaStream_t)stream));
   return MOE_OK;
 }
 

@@ -164,6 +164,26 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d, uint64_t a, uint64_t b, uin
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// MX block-scaled MMA (kind::mxf8f6f4, one E8M0 scale per 32 K-elements of
+// every row of A and of B): D[tmem] (+)= (A * SFA) * (B * SFB)^T.  sfa / sfb
+// are the TMEM addresses of the scale factors; their top two bits pick the
+// byte (the K-block of this MMA) inside each 32-bit TMEM word, and must
+// agree with the scale-factor ids in the instruction descriptor.
+__device__ __forceinline__ void mma_mx(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+// Copy a 32-row x 16-byte shared-memory block (descriptor sdesc) into TMEM
+// columns taddr..taddr+3 of lanes 0..31, replicated to all four 32-lane
+// quarters (the layout the block-scaled MMA reads its scale factors from).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // 32 lanes x 32 bit, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
@@ -192,6 +212,41 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;                 // layout: 128-byte swizzle
   return d;
+}
+
+// MX (OCP Microscaling) block scale: E8M0 code of a 32-element block whose
+// largest magnitude has the float bits amax_bits (non-negative, finite):
+// 127 + floor(log2 amax) - 8 (8 = exponent of E4M3's largest normal, 448 =
+// 1.75 * 2^8), clamped below at 0 (2^-127); 127 (X = 1) for an all-zero block.
+// A subnormal amax has exponent field 0 and clamps as floor(log2) would.
+__device__ __forceinline__ int mx_e8m0_code(uint32_t amax_bits) {
+  if (amax_bits == 0) return 127;
+  const int e = (int)(amax_bits >> 23) - 127;
+  return max(e - 8, -127) + 127;
+}
+// 1 / X = 2^-(code - 127) as a float: biased exponent 254 - code, in [8, 254]
+// for the codes mx_e8m0_code returns, so always an exact normal float.
+__device__ __forceinline__ float mx_inv_scale(int code) { return __uint_as_float((uint32_t)(254 - code) << 23); }
+
+// Shared-memory descriptor of an unswizzled K-major block of 8-row x 16-byte
+// core matrices stacked along the rows (16 bytes per row, 128 bytes per core
+// matrix): the source of tcgen05.cp's 32x128b shape.
+__device__ __forceinline__ uint64_t umma_desc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)(128 >> 4) << 32;        // stride byte offset: next 8 rows
+  d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
+  return d;                               // layout type 0: no swizzle
+}
+
+// Instruction descriptor of the block-scaled MMA (kind::mxf8f6f4, E8M0 scale
+// factors, fp32 accumulator, A/B K-major, shape M x N).  a_fmt / b_fmt: 0 =
+// E4M3, 5 = E2M1; sf_id: the byte of the scale-factor words this MMA uses
+// (for both A and B).
+__host__ __device__ __forceinline__ uint32_t umma_idesc_mx(int M, int N, uint32_t a_fmt, uint32_t b_fmt,
+                                                           uint32_t sf_id) {
+  return (sf_id << 4) | (a_fmt << 7) | (b_fmt << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24) | (sf_id << 29);
 }
 
 // Instruction descriptor: fp32 accumulator, A/B K-major, shape M x N.

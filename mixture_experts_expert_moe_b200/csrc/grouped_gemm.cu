@@ -40,6 +40,8 @@
 namespace moe {
 
 constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kGemmThreadsMx = 352; // + warp 10: MX activation scales
+constexpr int kSfChunk = 512;       // MX scale chunk: 128 rows x 4 K-blocks of E8M0
 constexpr int kWRows = 128;      // weight rows per tile = MMA M
 constexpr int kStageK = 128;     // bytes of K per stage (one swizzle row)
 constexpr int kWTileBytes = kWRows * kStageK;
@@ -154,17 +156,38 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
 // the token group has (rounded up to x_box).
 __device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// Shared-memory carve-up of the kernel (offsets from the 1024-aligned base).
+struct GemmSmem {
+  int stage_bytes;   // weights (two 128-row sub-tiles), token rows, MX: weight scale chunks
+  int sfb_bytes;     // MX: one token tile's activation scales for every stage
+  int nch;           // MX: 128-row chunks of the token tile
+};
+__host__ __device__ __forceinline__ GemmSmem gemm_smem_layout(int tn, int nk, bool mx) {
+  GemmSmem g;
+  g.nch = (tn + 127) / 128;
+  g.stage_bytes = 2 * kWTileBytes + tn * kStageK + (mx ? 2 * kSfChunk : 0);
+  g.sfb_bytes = mx ? nk * g.nch * kSfChunk : 0;
+  return g;
+}
+
+template <bool kMX>
+__global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int E = p.E;
+  // stages per tile and elements per stage along K: one 128-byte swizzle row
+  const bool byte_ops = kMX || p.fp8;
+  const int nk = p.K * (byte_ops ? 1 : 2) / kStageK;
+  const int k_elems = byte_ops ? kStageK : kStageK / 2;
   // every tile multiplies two 128-row weight sub-tiles with the same token
   // tile: gate and up rows (gate/up), or output rows n0 and n0+128 (down)
   const int w_bytes = 2 * kWTileBytes;
-  const int stage_bytes = w_bytes + p.tn * kStageK;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
+  const GemmSmem L = gemm_smem_layout(p.tn, nk, kMX);
+  const int stage_bytes = L.stage_bytes;
+  uint8_t* sfb_buf = smem + (size_t)p.stages * stage_bytes;             // MX: [2][sfb_bytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sfb_buf + 2 * (size_t)L.sfb_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + p.stages;
   uint64_t* acc_full = bars + 2 * p.stages;
@@ -172,7 +195,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint64_t* t_full = drain + 1;          // [kRing] a tile index was published
   uint64_t* t_empty = t_full + kRing;    // [kRing] every consumer has read it
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(t_empty + kRing);
+  uint64_t* sfb_full = t_empty + kRing;  // MX [2]: a tile's activation scales are staged
+  uint64_t* sfb_empty = sfb_full + 2;    // MX [2]: the MMAs that read them are done
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sfb_empty + 2);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
   int* s_drain_fail = s_abort + 1;   // a drain after an abort ran out of time
   int* s_ring = s_abort + 2;    // [kRing]
@@ -192,11 +217,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 8);
+      mbar_init(&sfb_full[a], 1);
+      mbar_init(&sfb_empty[a], 1);
     }
     mbar_init(drain, 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&t_full[r], 1);
-      mbar_init(&t_empty[r], 9);   // the MMA thread and the 8 epilogue warps
+      // the MMA thread, the 8 epilogue warps (and the MX scale warp)
+      mbar_init(&t_empty[r], kMX ? 10 : 9);
     }
     *s_abort = 0;
     *s_drain_fail = 0;
@@ -223,8 +251,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
-  const int nk = p.K * (p.fp8 ? 1 : 2) / kStageK;   // stages per tile
-  const int k_elems = p.fp8 ? kStageK : kStageK / 2; // elements per stage along K
   const int cols_per_acc = 2 * p.tn;
   const int xb = x_box_rows(p.tn);
   volatile int* abort_flag = s_abort;
@@ -266,7 +292,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           has1 = ti.wt * 2 * kWRows + kWRows < p.n_out;
         }
         const int nload = (ti.nrows + xb - 1) / xb;
-        const uint32_t tx = (has1 ? 2 : 1) * kWTileBytes + nload * xb * kStageK;
+        // a packed E2M1 weight box fills 16 KB of shared memory but completes
+        // only its 8 KB of codes as transaction bytes
+        const int w_tx = (kMX && p.w_fp4) ? kWTileBytes / 2 : kWTileBytes;
+        const uint32_t tx = (has1 ? 2 : 1) * (w_tx + (kMX ? kSfChunk : 0)) + nload * xb * kStageK;
         // weights streamed once (one token group) go first; re-read ones stay in L2
         const uint64_t pol_wt = s_groups[ti.e] > 1 ? pol_x : pol_w;
         for (int kb = 0; kb < nk; ++kb) {
@@ -281,6 +310,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (has1) tma_load_2d(sb + kWTileBytes, &tm_w, &full[stage], kc, row1, pol_wt);
           for (int l = 0; l < nload; ++l)
             tma_load_2d(sb + w_bytes + l * xb * kStageK, &tm_x, &full[stage], kc, ti.r0 + l * xb, pol_x);
+          if (kMX) {
+            // the weight sub-tiles' scale chunks (128 rows x 4 K-blocks, 512 bytes each)
+            uint8_t* sa = sb + w_bytes + p.tn * kStageK;
+            bulk_load(sa, p.w_sf + ((size_t)(row0 / kWRows) * nk + kb) * kSfChunk, kSfChunk, &full[stage]);
+            if (has1)
+              bulk_load(sa + kSfChunk, p.w_sf + ((size_t)(row1 / kWRows) * nk + kb) * kSfChunk, kSfChunk,
+                        &full[stage]);
+          }
           ++armed;
           if (++stage == p.stages) {
             stage = 0;
@@ -307,6 +344,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       const uint32_t fmt = p.fp8 ? 0u : 1u;
+      const uint32_t a_fmt_mx = p.w_fp4 ? 5u : 0u;   // E2M1 or E4M3 weights; activations E4M3
+      // MX scale factors in TMEM after the accumulators: weight sub-tiles 0/1, then the token tile
+      const uint32_t sf_col = tmem_base + (uint32_t)(p.n_acc * cols_per_acc);
       for (;; ++it) {
         const int slot = it % kRing;
         if (!wait_or_abort(&t_full[slot], (uint32_t)(it / kRing) & 1u, p.timeout_ns, abort_flag)) {
@@ -324,6 +364,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
+        const int sb_i = it & 1;
+        if (kMX && !wait_or_abort(&sfb_full[sb_i], (uint32_t)(it >> 1) & 1u, p.timeout_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * cols_per_acc);
         const uint32_t d1 = d0 + (uint32_t)p.tn;
@@ -338,15 +383,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t w0 = smem_u32(smem + (size_t)stage * stage_bytes);
           const uint32_t w1 = w0 + kWTileBytes;
           const uint32_t xa = w0 + (uint32_t)w_bytes;
+          if (kMX) {
+            // this stage's scale factors into TMEM (executed in order with the MMAs below)
+            const uint32_t sa = xa + (uint32_t)(p.tn * kStageK);
+            tmem_cp_32x128b_x4(sf_col, umma_desc_rows16(sa));
+            if (has1) tmem_cp_32x128b_x4(sf_col + 4, umma_desc_rows16(sa + kSfChunk));
+            const uint32_t sbf = smem_u32(sfb_buf + (size_t)sb_i * L.sfb_bytes) + (uint32_t)(kb * L.nch * kSfChunk);
+            for (int c = 0; c < L.nch; ++c)
+              tmem_cp_32x128b_x4(sf_col + 8 + 4 * c, umma_desc_rows16(sbf + c * kSfChunk));
+          }
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(xa + kk * 32);
             const uint32_t accum = (kb | kk) != 0;
-            if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
-            else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
-            if (has1) {
-              if (p.fp8) mma_e4m3(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
-              else mma_bf16(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
+            if (kMX) {
+              const uint32_t idx = umma_idesc_mx(kWRows, n_mma, a_fmt_mx, 0u, (uint32_t)kk);
+              const uint32_t sel = (uint32_t)kk << 30;     // byte kk of each scale word
+              mma_mx(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idx, sf_col | sel, (sf_col + 8) | sel, accum);
+              if (has1)
+                mma_mx(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idx, (sf_col + 4) | sel, (sf_col + 8) | sel,
+                       accum);
+            } else {
+              if (p.fp8) mma_e4m3(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
+              else mma_bf16(d0, umma_desc_sw128(w0 + kk * 32), bdesc, idesc, accum);
+              if (has1) {
+                if (p.fp8) mma_e4m3(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
+                else mma_bf16(d1, umma_desc_sw128(w1 + kk * 32), bdesc, idesc, accum);
+              }
             }
           }
           issued = true;
@@ -358,6 +421,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         tc_commit(&acc_full[acc]);
+        if (kMX) tc_commit(&sfb_empty[sb_i]);
       }
       if (!ok && issued) {
         // wait for the MMAs in flight before TMEM is freed
@@ -365,7 +429,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(drain, 0, kDrainTimeoutNs)) *s_drain_fail = 1;
       }
     }
-  } else {
+  } else if (warp < 10) {
     // ---------------- epilogue: warps 2..9 ----------------
     // two warps per TMEM lane quarter (a warp may only read lanes 32*(warp%4)..+31);
     // they take alternate 16-column chunks
@@ -411,7 +475,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uv = uv * sa * su;
               }
               const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;   // silu(g) * u
-              h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
+              if (kMX) {
+                // h rounded to bf16, then MX-quantised: the warp's 32 lanes hold the
+                // 32 consecutive features of one MX block of this row
+                const float hb = __bfloat162float(__float2bfloat16_rn(hv));
+                const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(hb) & 0x7FFFFFFFu);
+                const int code = mx_e8m0_code(amax);
+                const __nv_fp8_storage_t qv = __nv_cvt_float_to_fp8(hb * mx_inv_scale(code), __NV_SATFINITE,
+                                                                   __NV_E4M3);
+                reinterpret_cast<uint8_t*>(p.out)[(long long)row * p.n_out + n] = (uint8_t)qv;
+                if (lane == 0) p.h_sf[(long long)row * (p.n_out / 32) + (n >> 5)] = (uint8_t)code;
+              } else {
+                h[(long long)row * p.n_out + n] = __float2bfloat16_rn(hv);
+              }
             }
           }
         }
@@ -462,6 +538,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
+  } else if (kMX) {
+    // ---------------- MX scale warp (warp 10) ----------------
+    // Stages each token tile's activation scales (every stage, every
+    // 128-row chunk) in the layout tcgen05.cp reads: chunk byte
+    // (n % 32) * 16 + ((n % 128) / 32) * 4 + b holds row n's scale of K-block
+    // 4 * stage + b.  Rows past the tile get scale 1 (code 127).
+    const int kw = p.K / 128;    // scale words (4 K-blocks each) per row = stages
+    for (int it = 0;; ++it) {
+      const int slot = it % kRing;
+      if (!wait_or_abort(&t_full[slot], (uint32_t)(it / kRing) & 1u, p.timeout_ns, abort_flag)) break;
+      const int t = s_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[slot]);
+      if (t >= n_tiles) break;
+      const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
+      const int sb_i = it & 1;
+      if (!wait_or_abort(&sfb_empty[sb_i], ((uint32_t)(it >> 1) & 1u) ^ 1u, p.timeout_ns, abort_flag)) break;
+      uint32_t* buf = reinterpret_cast<uint32_t*>(sfb_buf + (size_t)sb_i * L.sfb_bytes);
+      for (int n = lane; n < L.nch * 128; n += 32) {
+        const int c = n >> 7, qq = (n >> 5) & 3, m0 = n & 31;
+        const uint32_t* src =
+            n < ti.nrows ? reinterpret_cast<const uint32_t*>(p.x_sf + (size_t)(ti.r0 + n) * (p.K / 32)) : nullptr;
+        uint32_t* dst = buf + c * (kSfChunk / 4) + m0 * 4 + qq;
+        for (int w = 0; w < kw; ++w) dst[w * L.nch * (kSfChunk / 4)] = src ? __ldg(src + w) : 0x7F7F7F7Fu;
+      }
+      fence_proxy_async();   // generic-proxy writes -> visible to tcgen05.cp (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfb_full[sb_i]);
+    }
   }
 
   __syncthreads();
@@ -494,55 +599,67 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D K-major tensor [rows, K] with a box of (128 bytes of K) x box_rows, 128-byte swizzle.
+// 2-D K-major tensor [rows, K] with a box of (128 bytes of K) x box_rows,
+// 128-byte swizzle.  elem_bytes 2: bf16; 1: one-byte codes; 0: E2M1 codes
+// packed two per byte in global memory, unpacked by TMA to one 16-byte chunk
+// per 16 elements (8 bytes of codes, 8 bytes of gap) in shared memory, the
+// operand layout of the block-scaled MMA for 4-bit A.
 static bool make_map(CUtensorMap* m, const void* base, long long rows, long long K, int elem_bytes,
                      int box_rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(K * elem_bytes)};
-  cuuint32_t box[2] = {(cuuint32_t)(kStageK / elem_bytes), (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(elem_bytes == 0 ? K / 2 : K * elem_bytes)};
+  cuuint32_t box[2] = {(cuuint32_t)(elem_bytes == 0 ? kStageK : kStageK / elem_bytes), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const CUtensorMapDataType dt = elem_bytes == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                   : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 
-size_t gemm_smem_bytes(int gateup, int tn, int stages, int E) {
-  const int stage_bytes = 2 * kWTileBytes + tn * kStageK;
-  (void)gateup;
-  return 1024 + (size_t)stages * stage_bytes + (2 * stages + 5 + 2 * kRing) * 8 + (kRing + 4) * 4 +
-         (size_t)(5 * E + 1) * 4;
+size_t gemm_smem_bytes(int tn, int stages, int E, int nk, bool mx) {
+  const GemmSmem L = gemm_smem_layout(tn, nk, mx);
+  return 1024 + (size_t)stages * L.stage_bytes + 2 * (size_t)L.sfb_bytes + (2 * stages + 9 + 2 * kRing) * 8 +
+         (kRing + 4) * 4 + (size_t)(5 * E + 1) * 4;
 }
 
-int gemm_pick_stages(int gateup, int tn, int E) {
+int gemm_pick_stages(int tn, int E, int nk, bool mx) {
   int s = 8;
-  while (s > 2 && gemm_smem_bytes(gateup, tn, s, E) > 225 * 1024) --s;
+  while (s > 2 && gemm_smem_bytes(tn, s, E, nk, mx) > 225 * 1024) --s;
   return s;
 }
 
 int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream) {
   GemmParams& p = L.p;
-  const int eb = p.fp8 ? 1 : 2;
+  const bool mx = p.mx != 0;
+  const int eb = (p.fp8 || mx) ? 1 : 2;
   CUtensorMap tw, tx;
-  if (!make_map(&tw, L.w, L.w_rows, p.K, eb, kWRows)) return -1;
+  if (!make_map(&tw, L.w, L.w_rows, p.K, mx && p.w_fp4 ? 0 : eb, kWRows)) return -1;
   if (!make_map(&tx, L.x, L.x_rows, p.K, eb, p.tn < 32 ? p.tn : 32)) return -1;
-  p.stages = gemm_pick_stages(p.gateup, p.tn, p.E);
+  const int nk = p.K * eb / kStageK;
+  p.stages = gemm_pick_stages(p.tn, p.E, nk, mx);
   const int cols = 2 * p.tn;
-  p.n_acc = 2 * cols <= 512 ? 2 : 1;
-  int need = p.n_acc * cols, alloc = 32;
+  const int sf_cols = mx ? 8 + 4 * ((p.tn + 127) / 128) : 0;   // MX scale factors after the accumulators
+  p.n_acc = 2 * cols + sf_cols <= 512 ? 2 : 1;
+  int need = p.n_acc * cols + sf_cols, alloc = 32;
   while (alloc < need) alloc <<= 1;
   p.tmem_cols = alloc;
-  const size_t smem = gemm_smem_bytes(p.gateup, p.tn, p.stages, p.E);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = gemm_smem_bytes(p.tn, p.stages, p.E, nk, mx);
+  const void* fn = mx ? (const void*)grouped_gemm_kernel<true> : (const void*)grouped_gemm_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  grouped_gemm_kernel<<<sms, kGemmThreads, smem, stream>>>(tw, tx, p);
+  if (mx)
+    grouped_gemm_kernel<true><<<sms, kGemmThreadsMx, smem, stream>>>(tw, tx, p);
+  else
+    grouped_gemm_kernel<false><<<sms, kGemmThreads, smem, stream>>>(tw, tx, p);
   return (int)cudaGetLastError();
 }
 

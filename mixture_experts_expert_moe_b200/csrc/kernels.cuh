@@ -61,6 +61,13 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
 // row r quantises token sorted[r] / k (zero codes, scale 1 for padding)
 cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
                               int nrows, int C, void* q, float* scale, int32_t* status, cudaStream_t s);
+// MXFP8 quantisation of bf16 rows of length C (C % 32 == 0): E4M3 codes
+// [rows, C] and E8M0 scales [rows, C/32]; rows and the row map as in
+// launch_quant_rows (padding rows: zero codes, scale code 127)
+cudaError_t launch_mx_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
+                                 int nrows, int C, void* codes, uint8_t* scales, cudaStream_t s);
+// per-row E8M0 scales [rows, K/32] -> tiled chunks (rows % 128 == 0, K % 128 == 0)
+cudaError_t launch_mx_tile_scales(const uint8_t* in, long long rows, int K, uint8_t* out, cudaStream_t s);
 cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s);
 cudaError_t launch_cast_bf16(const float* src, long long n, void* dst, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
@@ -110,6 +117,13 @@ struct GemmParams {
   int* tile_counter;     // next unclaimed tile of this launch (zero at launch)
   float* comb_out;       // down only, nullable: out32 [T, n_out] += comb_w[slot] * y instead of
   const float* comb_w;   //   writing y (top-k combine fused into the epilogue)
+  // MX block-scaled operands (kind::mxf8f6f4 with E8M0 scales per 32 K-elements;
+  // fp8 is 0 then, the scales are applied inside the MMA)
+  int mx;                // 1: MX operands
+  int w_fp4;             // MX weights are E2M1 codes packed two per byte (else E4M3)
+  const uint8_t* w_sf;   // weight scales in the tiled layout of moe_mx_tile_scales
+  const uint8_t* x_sf;   // activation scales [P, K/32]
+  uint8_t* h_sf;         // gate/up: out holds E4M3 codes of h [P, n_out], these their scales [P, n_out/32]
 };
 
 struct GemmLaunch {
@@ -120,8 +134,8 @@ struct GemmLaunch {
   GemmParams p;
 };
 
-size_t gemm_smem_bytes(int gateup, int tn, int stages, int E);
-int gemm_pick_stages(int gateup, int tn, int E);
+size_t gemm_smem_bytes(int tn, int stages, int E, int nk, bool mx);
+int gemm_pick_stages(int tn, int E, int nk, bool mx);
 // returns 0 on success, -1 if a tensor map could not be encoded, else a cudaError_t
 int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream);
 

@@ -14,8 +14,12 @@ def moe_flops(pairs: int, H: int, I: int) -> float:
     return 6.0 * pairs * H * I
 
 
-def expert_weight_bytes(H: int, I: int, a8w8: bool) -> int:
-    """Bytes of one expert's gate, up and down weights (+ fp32 channel scales)."""
+def expert_weight_bytes(H: int, I: int, a8w8: bool, mx: str = "") -> int:
+    """Bytes of one expert's gate, up and down weights: bf16; E4M3 + fp32
+    channel scales (a8w8); or MX codes (1 byte, or half a byte for E2M1) + one
+    E8M0 byte per 32 elements."""
+    if mx:
+        return 3 * H * I // (1 if mx == "mxfp8" else 2) + 3 * H * I // 32
     if a8w8:
         return 3 * H * I + 4 * (2 * I + H)
     return 2 * 3 * H * I
@@ -28,10 +32,10 @@ def tile_io_bytes(experts: int, m_tiles_per_expert: int, H: int, I: int,
 
 
 def layer_bytes(T: int, H: int, E: int, k: int, touched: int, I: int,
-                a8w8: bool, out_bytes: int = 2) -> int:
+                a8w8: bool, out_bytes: int = 2, mx: str = "") -> int:
     """Algorithmic bytes of one layer forward: touched experts' weights once,
     x read once, out written once, logits read, ids + weights written."""
-    return (touched * expert_weight_bytes(H, I, a8w8) + T * H * 2 + T * H * out_bytes
+    return (touched * expert_weight_bytes(H, I, a8w8, mx) + T * H * 2 + T * H * out_bytes
             + T * E * 4 + T * k * 8)
 
 
@@ -41,21 +45,28 @@ def align_bytes(n_slots: int, num_post: int, block_size: int) -> int:
     return 4 * n_slots + 4 * num_post + 4 * (num_post // block_size) + 4
 
 
-def gateup_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool) -> int:
+def _weight_matrix_bytes(rows: int, K: int, a8w8: bool, mx: str) -> int:
+    """Bytes of a [rows, K] weight matrix with its scales."""
+    if mx:
+        return rows * K // (1 if mx == "mxfp8" else 2) + rows * K // 32
+    if a8w8:
+        return rows * K + rows * 4
+    return rows * K * 2
+
+
+def gateup_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool, mx: str = "") -> int:
     """Algorithmic bytes of the gate/up GEMM launch: the touched experts' gate
-    and up weights once (+ fp32 channel scales in a8w8), the tokens' x once
-    (at the operand precision) and the routing it reads (one sorted slot id
-    per pair).  The permuted copy of x, h and padding are not counted."""
-    eb = 1 if a8w8 else 2
-    w = touched * (2 * I * H * eb + (2 * I * 4 if a8w8 else 0))
-    return w + T * H * eb + pairs * 4
+    and up weights once (+ their scales), the tokens' x once (at the operand
+    precision, one byte for FP8 and MX) and the routing it reads (one sorted
+    slot id per pair).  The permuted copy of x, h and padding are not
+    counted."""
+    eb = 1 if (a8w8 or mx) else 2
+    return touched * _weight_matrix_bytes(2 * I, H, a8w8, mx) + T * H * eb + pairs * 4
 
 
-def down_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool) -> int:
+def down_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bool, mx: str = "") -> int:
     """Algorithmic bytes of the down GEMM launch: the touched experts' down
-    weights once (+ fp32 channel scales in a8w8), the fp32 token outputs
-    written once and the routing it reads (slot id and weight per pair).
-    The h operand and padding are not counted."""
-    eb = 1 if a8w8 else 2
-    w = touched * (H * I * eb + (H * 4 if a8w8 else 0))
-    return w + T * H * 4 + pairs * 8
+    weights once (+ their scales), the fp32 token outputs written once and the
+    routing it reads (slot id and weight per pair).  The h operand and
+    padding are not counted."""
+    return touched * _weight_matrix_bytes(H, I, a8w8, mx) + T * H * 4 + pairs * 8

@@ -54,6 +54,7 @@ class MoEConfig:
     seed: int = SEED_BASE
     n_shared: int = 0           # always-on shared experts stored after the E routed ones
     bias_mode: str = "logits"   # "logits": bias feeds selection and weights; "select": selection only
+    mx: str = ""                # "mxfp8" / "mxfp4": MX block-scaled weights drawn as codes + scales
 
     def with_(self, **kw) -> "MoEConfig":
         return replace(self, **kw)
@@ -79,6 +80,10 @@ CONFIGS = {
     "decode": MoEConfig("decode", T=64, H=7168, I=2048, E=256, k=8, bm=16,
                         a8w8=True, seed=SEED_BASE + 4),
 }
+
+# E8M0 scale code around which MX weight scales are drawn (codes uniform over
+# E4M3 have an rms near 100, over E2M1 near 3)
+MX_SCALE_CODE = {"mxfp8": 114, "mxfp4": 119}
 
 ALIGN_CONFIG = dict(T=16384, E=256, k=8, bm=64, zipf_s=1.0, seed=SEED_BASE + 1)
 
@@ -109,24 +114,48 @@ def fp8_weights(E, rows, cols, std, seed, device="cpu"):
     return codes, scales
 
 
-def mx_weights(E, rows, cols, elem, seed, scale_code_mean=122):
+def mx_weights(E, rows, cols, elem, seed, scale_code_mean=122, device=None):
     """MX block-scaled weights drawn directly (no quantisation step): uint8
     element codes [E, rows, cols] uniform over the finite codes of `elem`
     ("e2m1": 4-bit codes 0..15; "e4m3": the E4M3FN codes except NaN), and
     E8M0 scale codes [E, rows, cols/32] = scale_code_mean + {-1, 0, +1}
-    (powers of two around 2^(mean-127))."""
+    (powers of two around 2^(mean-127)).
+
+    device None: numpy arrays from a numpy generator; a torch device: uint8
+    tensors drawn there by a seeded torch generator (for large layers; the
+    two paths draw different, equally distributed values)."""
     if cols % 32:
         raise ValueError("cols must be a multiple of 32")
+    if elem not in ("e2m1", "e4m3"):
+        raise ValueError(elem)
+    if device is not None:
+        g = _gen(device, seed)
+        hi = 16 if elem == "e2m1" else 255
+        codes = torch.randint(0, hi, (E, rows, cols), generator=g, device=device, dtype=torch.uint8)
+        if elem == "e4m3":
+            codes[(codes & 0x7F) == 0x7F] = 0          # no NaN codes
+        off = torch.randint(-1, 2, (E, rows, cols // 32), generator=g, device=device, dtype=torch.int32)
+        return codes, (scale_code_mean + off).to(torch.uint8)
     rng = np.random.default_rng(seed)
     if elem == "e2m1":
         codes = rng.integers(0, 16, size=(E, rows, cols), dtype=np.uint8)
-    elif elem == "e4m3":
+    else:
         codes = rng.integers(0, 255, size=(E, rows, cols), dtype=np.uint8)
         codes[(codes & 0x7F) == 0x7F] = 0          # no NaN codes
-    else:
-        raise ValueError(elem)
     scales = (scale_code_mean + rng.integers(-1, 2, size=(E, rows, cols // 32))).astype(np.uint8)
     return codes, scales
+
+
+def pack_e2m1(codes):
+    """E2M1 codes (uint8 values 0..15) [..., K] packed two per byte [..., K/2]:
+    element 2j in the low nibble, 2j+1 in the high nibble (the layout the MX
+    kernels read; packing only moves bits).  numpy array or torch tensor."""
+    if codes.shape[-1] % 2:
+        raise ValueError("K must be even")
+    if isinstance(codes, torch.Tensor):
+        return ((codes[..., 0::2] & 0xF) | ((codes[..., 1::2] & 0xF) << 4)).contiguous()
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[..., 0::2] & 0xF) | ((codes[..., 1::2] & 0xF) << 4)
 
 
 def make_layer(cfg: MoEConfig, device="cpu", weights=True):
@@ -149,7 +178,14 @@ def make_layer(cfg: MoEConfig, device="cpu", weights=True):
         d["logits"] = normal((T, E), 1.0, s * 16 + 3, device)
     d["bias"] = normal((E,), 1.0, s * 16 + 4, device) if cfg.bias else None
     if weights:
-        if cfg.a8w8:
+        if cfg.mx:
+            # MX weights drawn directly as codes + E8M0 scales, scale codes
+            # chosen so the layer's outputs are of order 0.1..1 at hidden 7168
+            elem = "e2m1" if cfg.mx == "mxfp4" else "e4m3"
+            mean = MX_SCALE_CODE[cfg.mx]
+            d["w13_codes"], d["w13_sf"] = mx_weights(EW, 2 * I, H, elem, s * 16 + 7, mean, device=device)
+            d["w2_codes"], d["w2_sf"] = mx_weights(EW, H, I, elem, s * 16 + 8, mean, device=device)
+        elif cfg.a8w8:
             d["w13_q"], d["w13_s"] = fp8_weights(EW, 2 * I, H, 0.02, s * 16 + 5, device)
             d["w2_q"], d["w2_s"] = fp8_weights(EW, H, I, 0.02, s * 16 + 6, device)
         else:

@@ -56,15 +56,24 @@ MX_BLOCK = 32
 # ---------------------------------------------------------------------------
 
 
-def e2m1_decode(codes) -> np.ndarray:
+def _e2m1_formula(c) -> np.ndarray:
     """Value of E2M1 codes (low 4 bits): sign bit 3, exponent bits 2..1
     (bias 1), mantissa bit 0; exponent 0 is subnormal (0 or 0.5)."""
-    c = np.asarray(codes).astype(np.int64) & 0xF
+    c = np.asarray(c).astype(np.int64) & 0xF
     sign = np.where(c & 0x8, -1.0, 1.0)
     e = (c >> 1) & 0x3
     m = c & 0x1
     mag = np.where(e == 0, m * 0.5, (1.0 + 0.5 * m) * np.power(2.0, e - 1))
     return sign * mag
+
+
+# the formula evaluated once for every byte value (only the low 4 bits count)
+_E2M1_TABLE = _e2m1_formula(np.arange(256))
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """Value of E2M1 codes (the formula of ``_e2m1_formula``, looked up)."""
+    return _E2M1_TABLE[np.asarray(codes).astype(np.uint8, copy=False)]
 
 
 def e2m1_values() -> np.ndarray:

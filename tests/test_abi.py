@@ -31,7 +31,7 @@ def test_status_strings_and_version():
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
     assert lib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
-    assert lib.moe_version() == m.ABI_VERSION == 200
+    assert lib.moe_version() == m.ABI_VERSION == 300
 
 
 def test_align_sizes():
@@ -209,3 +209,43 @@ def test_forward_workspace_follows_the_combine_rule():
     assert _fwd_ws(k=2, out_dtype=0) == _fwd_ws(k=2, out_dtype=2)
     # a shared expert counts as a slot: k = 3 + 1 shared is fused as well
     assert _fwd_ws(k=3, n_shared=1, out_dtype=0) - _fwd_ws(k=3, n_shared=1, out_dtype=2) == T * H * 4
+
+
+# ---------------------------------------------------------------------------
+# MX block-scaled weights (MOE_MXFP8 = 3, MOE_MXFP4 = 4)
+# ---------------------------------------------------------------------------
+def test_mx_workspace_and_tile_limit():
+    lib = m.load_library()
+    n16, n8, nmx = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn()), ctypes.byref(n16)) == 0
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=3)), ctypes.byref(nmx)) == 0
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=4)), ctypes.byref(n8)) == 0
+    assert n8.value == nmx.value < n16.value        # one-byte activations, no bf16 copy of h
+    # MX token tiles hold at most 128 tokens
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=3, tile_tokens=256)), ctypes.byref(n8)) == 2
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=3, tile_tokens=128)), ctypes.byref(n8)) == 0
+    assert lib.moe_ffn_workspace(ctypes.byref(_ffn(wdtype=5)), ctypes.byref(n8)) == 1
+
+
+def test_mx_forward_needs_its_scales_and_alignment():
+    lib = m.load_library()
+    ws = ctypes.c_void_p(_ADDR)
+    # MX weights without their tiled scales
+    assert lib.moe_forward(ctypes.byref(_fwd(wdtype=3)), ws, 1 << 40, None, None) == 1
+    assert lib.moe_forward(ctypes.byref(_fwd(wdtype=4, w13_mx_scale=_ADDR)), ws, 1 << 40, None, None) == 1
+    # packed E2M1 weights need 32-byte aligned bases (the 4-bit tensor maps' rule)
+    a32 = (_ADDR + 31) // 32 * 32
+    bad = _fwd(wdtype=4, w13=a32 + 16, w2=a32, w13_mx_scale=_ADDR, w2_mx_scale=_ADDR)
+    assert lib.moe_forward(ctypes.byref(bad), ws, 1 << 40, None, None) == 1
+
+
+def test_mx_helpers_argument_errors():
+    lib = m.load_library()
+    p = ctypes.c_void_p(_ADDR)
+    assert lib.moe_mx_tile_scales(p, 100, 256, p, None) == 1       # rows % 128
+    assert lib.moe_mx_tile_scales(p, 128, 96, p, None) == 1        # K % 128
+    assert lib.moe_mx_tile_scales(None, 128, 256, p, None) == 1
+    assert lib.moe_mx_tile_scales(p, 0, 256, p, None) == 0         # nothing to do
+    assert lib.moe_mx_quantize_rows(p, 4, 48, p, p, None) == 1     # C % 32
+    assert lib.moe_mx_quantize_rows(p, -1, 64, p, p, None) == 1
+    assert lib.moe_mx_quantize_rows(p, 0, 64, p, p, None) == 0

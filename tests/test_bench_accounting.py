@@ -70,3 +70,14 @@ def test_traffic_lookup_needs_matching_source(tmp_path):
 @pytest.mark.parametrize("world,units,steps,ms", [(1, 2048, 100, 400.0), (8, 2048, 50, 210.0)])
 def test_job_throughput(world, units, steps, ms):
     assert bench.job_throughput(world, units, steps, ms) == pytest.approx(world * units * steps / (ms / 1000))
+
+
+def test_mx_weight_bytes_by_hand():
+    from mixture_experts_expert_moe_b200.roofline import expert_weight_bytes
+    H, I = 256, 128
+    # E2M1 codes at half a byte, E4M3 at one, plus one E8M0 byte per 32 elements
+    assert expert_weight_bytes(H, I, False, "mxfp4") == 3 * H * I // 2 + 3 * H * I // 32
+    assert expert_weight_bytes(H, I, False, "mxfp8") == 3 * H * I + 3 * H * I // 32
+    cfg = MoEConfig("t", T=4, H=H, I=I, E=8, k=2, bm=16, mx="mxfp4")
+    assert bench.gateup_bytes(cfg, 3) == 3 * (2 * I * H // 2 + 2 * I * H // 32) + 4 * H + 8 * 4
+    assert bench.down_bytes(cfg, 3) == 3 * (H * I // 2 + H * I // 32) + 4 * H * 4 + 8 * 8

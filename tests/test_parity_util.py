@@ -22,3 +22,17 @@ def test_cover_sample_reaches_every_expert_and_the_hot_tails():
 def test_cover_sample_single_token():
     toks, reached, touched = cover_sample(np.array([[3, 1, 2]]))
     assert list(toks) == [0] and reached == touched == 3
+
+
+def test_pack_e2m1_layout_numpy_and_torch():
+    import torch
+    from moe_inputs import mx_weights, pack_e2m1
+    codes, scales = mx_weights(2, 4, 64, "e2m1", seed=3)
+    p = pack_e2m1(codes)
+    assert p.shape == (2, 4, 32)
+    assert np.array_equal(p & 0xF, codes[..., 0::2]) and np.array_equal(p >> 4, codes[..., 1::2])
+    assert np.array_equal(pack_e2m1(torch.from_numpy(codes)).numpy(), p)
+    tc, ts = mx_weights(2, 4, 64, "e4m3", seed=3, device="cpu")
+    assert tc.dtype == torch.uint8 and ts.shape == (2, 4, 2)
+    assert not bool(((tc & 0x7F) == 0x7F).any())        # no NaN codes
+    assert int(ts.min()) >= 121 and int(ts.max()) <= 123
