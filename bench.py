@@ -137,6 +137,8 @@ def build_layer(m, cfg, dev, out_dtype=torch.bfloat16, tile_tokens=0, data=None)
         pack = pack_e2m1 if cfg.mx == "mxfp4" else (lambda c: c)
         w13, w2 = pack(d["w13_codes"]), pack(d["w2_codes"])
         s13, s2 = m.mx_tile_scales(d["w13_sf"]), m.mx_tile_scales(d["w2_sf"])
+        for key in ("w13_codes", "w2_codes", "w13_sf", "w2_sf"):    # the packed / tiled copies replace them
+            del d[key]
         layer = m.MoELayer(w13, w2, cfg.k, cfg.bm, out_dtype=out_dtype, tile_tokens=tile_tokens,
                            n_shared=cfg.n_shared, bias_mode=cfg.bias_mode, mx=cfg.mx, w13_mx_scale=s13,
                            w2_mx_scale=s2)

@@ -156,17 +156,19 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, lo
 // the token group has (rounded up to x_box).
 __device__ __forceinline__ int x_box_rows(int tn) { return tn < 32 ? tn : 32; }
 
-// Shared-memory carve-up of the kernel (offsets from the 1024-aligned base).
+// Shared-memory carve-up of one pipeline stage: two 128-row weight sub-tiles,
+// the token rows, and with MX operands the weight sub-tiles' scale chunks and
+// the token rows' scale chunks (stages stay 1024-byte aligned for the
+// 128-byte swizzle).
 struct GemmSmem {
-  int stage_bytes;   // weights (two 128-row sub-tiles), token rows, MX: weight scale chunks
-  int sfb_bytes;     // MX: one token tile's activation scales for every stage
-  int nch;           // MX: 128-row chunks of the token tile
+  int stage_bytes;
+  int nch;           // MX: 128-row scale chunks of the token tile
 };
-__host__ __device__ __forceinline__ GemmSmem gemm_smem_layout(int tn, int nk, bool mx) {
+__host__ __device__ __forceinline__ GemmSmem gemm_smem_layout(int tn, bool mx) {
   GemmSmem g;
   g.nch = (tn + 127) / 128;
-  g.stage_bytes = 2 * kWTileBytes + tn * kStageK + (mx ? 2 * kSfChunk : 0);
-  g.sfb_bytes = mx ? nk * g.nch * kSfChunk : 0;
+  const int b = 2 * kWTileBytes + tn * kStageK + (mx ? (2 + g.nch) * kSfChunk : 0);
+  g.stage_bytes = (b + 1023) / 1024 * 1024;
   return g;
 }
 
@@ -184,10 +186,10 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
   // every tile multiplies two 128-row weight sub-tiles with the same token
   // tile: gate and up rows (gate/up), or output rows n0 and n0+128 (down)
   const int w_bytes = 2 * kWTileBytes;
-  const GemmSmem L = gemm_smem_layout(p.tn, nk, kMX);
+  const GemmSmem L = gemm_smem_layout(p.tn, kMX);
   const int stage_bytes = L.stage_bytes;
-  uint8_t* sfb_buf = smem + (size_t)p.stages * stage_bytes;             // MX: [2][sfb_bytes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sfb_buf + 2 * (size_t)L.sfb_bytes);
+  const int sf_off = w_bytes + p.tn * kStageK;    // MX: weight scale chunks, then token scale chunks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * stage_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + p.stages;
   uint64_t* acc_full = bars + 2 * p.stages;
@@ -195,9 +197,7 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint64_t* t_full = drain + 1;          // [kRing] a tile index was published
   uint64_t* t_empty = t_full + kRing;    // [kRing] every consumer has read it
-  uint64_t* sfb_full = t_empty + kRing;  // MX [2]: a tile's activation scales are staged
-  uint64_t* sfb_empty = sfb_full + 2;    // MX [2]: the MMAs that read them are done
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sfb_empty + 2);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(t_empty + kRing);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
   int* s_drain_fail = s_abort + 1;   // a drain after an abort ran out of time
   int* s_ring = s_abort + 2;    // [kRing]
@@ -211,14 +211,13 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < p.stages; ++s) {
-      mbar_init(&full[s], 1);
+      // MX: the 32 lanes of the scale warp also arrive, once their copies land
+      mbar_init(&full[s], kMX ? 33 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 8);
-      mbar_init(&sfb_full[a], 1);
-      mbar_init(&sfb_empty[a], 1);
     }
     mbar_init(drain, 1);
     for (int r = 0; r < kRing; ++r) {
@@ -312,7 +311,7 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
             tma_load_2d(sb + w_bytes + l * xb * kStageK, &tm_x, &full[stage], kc, ti.r0 + l * xb, pol_x);
           if (kMX) {
             // the weight sub-tiles' scale chunks (128 rows x 4 K-blocks, 512 bytes each)
-            uint8_t* sa = sb + w_bytes + p.tn * kStageK;
+            uint8_t* sa = sb + sf_off;
             bulk_load(sa, p.w_sf + ((size_t)(row0 / kWRows) * nk + kb) * kSfChunk, kSfChunk, &full[stage]);
             if (has1)
               bulk_load(sa + kSfChunk, p.w_sf + ((size_t)(row1 / kWRows) * nk + kb) * kSfChunk, kSfChunk,
@@ -364,11 +363,6 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
           ok = false;
           break;
         }
-        const int sb_i = it & 1;
-        if (kMX && !wait_or_abort(&sfb_full[sb_i], (uint32_t)(it >> 1) & 1u, p.timeout_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * cols_per_acc);
         const uint32_t d1 = d0 + (uint32_t)p.tn;
@@ -385,12 +379,11 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
           const uint32_t xa = w0 + (uint32_t)w_bytes;
           if (kMX) {
             // this stage's scale factors into TMEM (executed in order with the MMAs below)
-            const uint32_t sa = xa + (uint32_t)(p.tn * kStageK);
+            const uint32_t sa = w0 + (uint32_t)sf_off;
             tmem_cp_32x128b_x4(sf_col, umma_desc_rows16(sa));
             if (has1) tmem_cp_32x128b_x4(sf_col + 4, umma_desc_rows16(sa + kSfChunk));
-            const uint32_t sbf = smem_u32(sfb_buf + (size_t)sb_i * L.sfb_bytes) + (uint32_t)(kb * L.nch * kSfChunk);
             for (int c = 0; c < L.nch; ++c)
-              tmem_cp_32x128b_x4(sf_col + 8 + 4 * c, umma_desc_rows16(sbf + c * kSfChunk));
+              tmem_cp_32x128b_x4(sf_col + 8 + 4 * c, umma_desc_rows16(sa + (2 + c) * kSfChunk));
           }
 #pragma unroll
           for (int kk = 0; kk < kStageK / 32; ++kk) {
@@ -421,7 +414,6 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
         }
         if (!ok) break;
         tc_commit(&acc_full[acc]);
-        if (kMX) tc_commit(&sfb_empty[sb_i]);
       }
       if (!ok && issued) {
         // wait for the MMAs in flight before TMEM is freed
@@ -540,11 +532,16 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
     }
   } else if (kMX) {
     // ---------------- MX scale warp (warp 10) ----------------
-    // Stages each token tile's activation scales (every stage, every
-    // 128-row chunk) in the layout tcgen05.cp reads: chunk byte
-    // (n % 32) * 16 + ((n % 128) / 32) * 4 + b holds row n's scale of K-block
-    // 4 * stage + b.  Rows past the tile get scale 1 (code 127).
-    const int kw = p.K / 128;    // scale words (4 K-blocks each) per row = stages
+    // For every stage the producer fills, copies the token rows' scales of
+    // its 4 K-blocks (one 32-bit word per row) into the stage's token scale
+    // chunks, in the layout tcgen05.cp reads: chunk c, byte
+    // (n % 32) * 16 + ((n % 128) / 32) * 4 + b holds row 128c + n's scale of
+    // K-block 4 * stage + b.  The copies are cp.async (fire and forget); each
+    // lane's arrive on the stage's full barrier fires when its copies have
+    // landed.  Rows past the token group are not written: the MMA columns
+    // they scale are never read.
+    int stage = 0;
+    uint32_t phase = 0;
     for (int it = 0;; ++it) {
       const int slot = it % kRing;
       if (!wait_or_abort(&t_full[slot], (uint32_t)(it / kRing) & 1u, p.timeout_ns, abort_flag)) break;
@@ -553,20 +550,26 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
       if (lane == 0) mbar_arrive(&t_empty[slot]);
       if (t >= n_tiles) break;
       const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
-      const int sb_i = it & 1;
-      if (!wait_or_abort(&sfb_empty[sb_i], ((uint32_t)(it >> 1) & 1u) ^ 1u, p.timeout_ns, abort_flag)) break;
-      uint32_t* buf = reinterpret_cast<uint32_t*>(sfb_buf + (size_t)sb_i * L.sfb_bytes);
-      for (int n = lane; n < L.nch * 128; n += 32) {
-        const int c = n >> 7, qq = (n >> 5) & 3, m0 = n & 31;
-        const uint32_t* src =
-            n < ti.nrows ? reinterpret_cast<const uint32_t*>(p.x_sf + (size_t)(ti.r0 + n) * (p.K / 32)) : nullptr;
-        uint32_t* dst = buf + c * (kSfChunk / 4) + m0 * 4 + qq;
-        for (int w = 0; w < kw; ++w) dst[w * L.nch * (kSfChunk / 4)] = src ? __ldg(src + w) : 0x7F7F7F7Fu;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_or_abort(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = smem_u32(smem + (size_t)stage * stage_bytes + sf_off + 2 * kSfChunk);
+        for (int n = lane; n < ti.nrows; n += 32) {
+          const uint32_t off = (uint32_t)((n >> 7) * kSfChunk + (n & 31) * 16 + ((n >> 5) & 3) * 4);
+          cp_async_4(dst + off, p.x_sf + (size_t)(ti.r0 + n) * (p.K / 32) + (size_t)kb * 4);
+        }
+        cp_async_mbar_arrive_noinc(&full[stage]);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
-      fence_proxy_async();   // generic-proxy writes -> visible to tcgen05.cp (async proxy)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sfb_full[sb_i]);
+      if (!ok) break;
     }
+    cp_async_wait_all();   // no copy of this warp may land after the CTA exits
   }
 
   __syncthreads();
@@ -622,15 +625,15 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, long long
 }
 
 
-size_t gemm_smem_bytes(int tn, int stages, int E, int nk, bool mx) {
-  const GemmSmem L = gemm_smem_layout(tn, nk, mx);
-  return 1024 + (size_t)stages * L.stage_bytes + 2 * (size_t)L.sfb_bytes + (2 * stages + 9 + 2 * kRing) * 8 +
-         (kRing + 4) * 4 + (size_t)(5 * E + 1) * 4;
+size_t gemm_smem_bytes(int tn, int stages, int E, bool mx) {
+  const GemmSmem L = gemm_smem_layout(tn, mx);
+  return 1024 + (size_t)stages * L.stage_bytes + (2 * stages + 5 + 2 * kRing) * 8 + (kRing + 4) * 4 +
+         (size_t)(5 * E + 1) * 4;
 }
 
-int gemm_pick_stages(int tn, int E, int nk, bool mx) {
+int gemm_pick_stages(int tn, int E, bool mx) {
   int s = 8;
-  while (s > 2 && gemm_smem_bytes(tn, s, E, nk, mx) > 225 * 1024) --s;
+  while (s > 2 && gemm_smem_bytes(tn, s, E, mx) > 225 * 1024) --s;
   return s;
 }
 
@@ -641,15 +644,14 @@ int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream) {
   CUtensorMap tw, tx;
   if (!make_map(&tw, L.w, L.w_rows, p.K, mx && p.w_fp4 ? 0 : eb, kWRows)) return -1;
   if (!make_map(&tx, L.x, L.x_rows, p.K, eb, p.tn < 32 ? p.tn : 32)) return -1;
-  const int nk = p.K * eb / kStageK;
-  p.stages = gemm_pick_stages(p.tn, p.E, nk, mx);
+  p.stages = gemm_pick_stages(p.tn, p.E, mx);
   const int cols = 2 * p.tn;
   const int sf_cols = mx ? 8 + 4 * ((p.tn + 127) / 128) : 0;   // MX scale factors after the accumulators
   p.n_acc = 2 * cols + sf_cols <= 512 ? 2 : 1;
   int need = p.n_acc * cols + sf_cols, alloc = 32;
   while (alloc < need) alloc <<= 1;
   p.tmem_cols = alloc;
-  const size_t smem = gemm_smem_bytes(p.tn, p.stages, p.E, nk, mx);
+  const size_t smem = gemm_smem_bytes(p.tn, p.stages, p.E, mx);
   const void* fn = mx ? (const void*)grouped_gemm_kernel<true> : (const void*)grouped_gemm_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;

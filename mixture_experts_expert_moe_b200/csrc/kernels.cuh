@@ -134,8 +134,8 @@ struct GemmLaunch {
   GemmParams p;
 };
 
-size_t gemm_smem_bytes(int tn, int stages, int E, int nk, bool mx);
-int gemm_pick_stages(int tn, int E, int nk, bool mx);
+size_t gemm_smem_bytes(int tn, int stages, int E, bool mx);
+int gemm_pick_stages(int tn, int E, bool mx);
 // returns 0 on success, -1 if a tensor map could not be encoded, else a cudaError_t
 int launch_grouped_gemm(GemmLaunch& L, cudaStream_t stream);
 
