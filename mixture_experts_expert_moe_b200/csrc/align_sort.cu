@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
       const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
       r.plan[plan_start(E) + e] = s_off[e];
       r.plan[plan_rows(E) + e] = rows;
+      r.plan[plan_real(E) + e] = s_tot[e];
       s_g[e] = (rows + r.tn - 1) / r.tn;
     }
     __syncthreads();

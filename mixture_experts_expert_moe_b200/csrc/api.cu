@@ -232,8 +232,8 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   const int R = (int)s.rows_max;   // grid size of the row kernels (they read num_post on the device)
 
   if (!plan_ready)
-    MOE_CU(moe::launch_plan(expert_ids, num_post, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan, status,
-                            stream));
+    MOE_CU(moe::launch_plan(expert_ids, num_post, sorted, N, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan,
+                            status, stream));
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
   if (s.mx) {
     // every sorted row MX-quantises its token (codes + a scale per 32 elements)

@@ -53,9 +53,10 @@ constexpr long long kDrainTimeoutNs = 100000000LL;
 // Tile plan for the stand-alone FFN (moe_grouped_ffn), from the align & sort
 // outputs; layout in kernels.cuh, ordering in plan.cuh.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ expert_ids,
-                                                    const int32_t* __restrict__ num_post, int P, int E, int bm,
-                                                    int tn, int nw_gu, int nw_dn, int32_t* __restrict__ plan,
-                                                    int32_t* status) {
+                                                    const int32_t* __restrict__ num_post,
+                                                    const int32_t* __restrict__ sorted, int N, int P, int E,
+                                                    int bm, int tn, int nw_gu, int nw_dn,
+                                                    int32_t* __restrict__ plan, int32_t* status) {
   extern __shared__ int sm[];
   int* s_first = sm;        // [E] first block of expert
   int* s_nblk = sm + E;     // [E] blocks of expert -> token groups
@@ -84,18 +85,26 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
     const int rows = s_nblk[e] * bm;
-    plan[plan_start(E) + e] = s_first[e] * bm;
+    const int start = s_first[e] * bm;
+    // padding (slot id >= N) fills the end of the segment: count it in the last block
+    int real = rows;
+    for (int i = rows - 1; i >= 0 && i >= rows - bm; --i) {
+      if (sorted[start + i] < N) break;
+      --real;
+    }
+    plan[plan_start(E) + e] = start;
     plan[plan_rows(E) + e] = rows;
+    plan[plan_real(E) + e] = real;
     s_nblk[e] = (rows + tn - 1) / tn;
   }
   __syncthreads();
   finish_plan(plan, s_nblk, E, nw_gu, nw_dn, tn, np, sc);
 }
 
-cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
-                        int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s) {
-  plan_kernel<<<1, 1024, (5 * E + 2) * sizeof(int), s>>>(expert_ids, num_post, P, E, bm, tn, nw_gu, nw_dn, plan,
-                                                         status);
+cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, const int32_t* sorted, int N, int P,
+                        int E, int bm, int tn, int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s) {
+  plan_kernel<<<1, 1024, (5 * E + 2) * sizeof(int), s>>>(expert_ids, num_post, sorted, N, P, E, bm, tn, nw_gu,
+                                                         nw_dn, plan, status);
   return cudaGetLastError();
 }
 
@@ -106,6 +115,9 @@ struct TileInfo {
 
 // Tile t of the list: the list position of its expert (last position whose
 // tile range starts at or before t), then weight tile and token group.
+// nrows counts the group's real rows only (the expert's padding rows, at the
+// end of its segment, are neither loaded nor multiplied); a group of padding
+// alone keeps one row, which every epilogue skips as padding.
 __device__ __forceinline__ TileInfo decode_tile(int t, const int* s_pref, const int* s_perm, const int* s_start,
                                                 const int* s_rows, const int* s_groups, int E, int tn) {
   int lo = 0, hi = E - 1;
@@ -120,7 +132,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const int* s_pref, const 
   ti.wt = local / G;
   const int g = local - ti.wt * G;
   ti.r0 = s_start[ti.e] + g * tn;
-  ti.nrows = min(tn, s_rows[ti.e] - g * tn);
+  ti.nrows = max(1, min(tn, s_rows[ti.e] - g * tn));
   return ti;
 }
 
@@ -238,7 +250,7 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
   const int pref_off = plan_pref(E, p.gateup != 0);
   for (int i = threadIdx.x; i < E; i += blockDim.x) {
     s_start[i] = p.plan[plan_start(E) + i];
-    s_rows[i] = p.plan[plan_rows(E) + i];
+    s_rows[i] = p.plan[plan_real(E) + i];     // real rows per expert (padding excluded)
     s_groups[i] = p.plan[plan_groups(E) + i];
     s_perm[i] = p.plan[plan_perm(E) + i];
   }

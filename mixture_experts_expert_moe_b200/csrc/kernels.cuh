@@ -78,22 +78,25 @@ cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, 
 //   [4] gate/up tiles of the hot experts  [5] down tiles of the hot experts
 //   [6] gate/up tile counter  [7] down tile counter (zeroed by the writer,
 //       advanced by the GEMM launches as they claim tiles)
-//   seg_start[E] @8, seg_rows[E] @8+E, groups[E] @8+2E (by expert),
+//   seg_start[E] @8, seg_rows[E] @8+E (padded), groups[E] @8+2E (by expert),
 //   perm[E] @8+3E (expert at each list position: hot experts first),
-//   pref_gu[E+1] @8+4E, pref_dn[E+1] @9+5E (tile prefix by list position)
+//   pref_gu[E+1] @8+4E, pref_dn[E+1] @9+5E (tile prefix by list position),
+//   seg_real[E] @10+6E (slots of the expert: its segment's rows that are not
+//   padding, which come first in the segment)
 enum {
   PLAN_TILES_GU = 0, PLAN_TILES_DN = 1, PLAN_TN = 2, PLAN_NUM_POST = 3, PLAN_HOT_GU = 4, PLAN_HOT_DN = 5,
   PLAN_COUNTER_GU = 6, PLAN_COUNTER_DN = 7, PLAN_HEADER = 8
 };
-__host__ __device__ inline int plan_ints(int E) { return 10 + 6 * E; }
+__host__ __device__ inline int plan_ints(int E) { return 10 + 7 * E; }
 __host__ __device__ inline int plan_start(int) { return PLAN_HEADER; }
 __host__ __device__ inline int plan_rows(int E) { return PLAN_HEADER + E; }
 __host__ __device__ inline int plan_groups(int E) { return PLAN_HEADER + 2 * E; }
 __host__ __device__ inline int plan_perm(int E) { return PLAN_HEADER + 3 * E; }
 __host__ __device__ inline int plan_pref(int E, bool gateup) { return gateup ? PLAN_HEADER + 4 * E : PLAN_HEADER + 5 * E + 1; }
+__host__ __device__ inline int plan_real(int E) { return PLAN_HEADER + 6 * E + 2; }
 __host__ __device__ inline int plan_counter(int, bool gateup) { return gateup ? PLAN_COUNTER_GU : PLAN_COUNTER_DN; }
-cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, int P, int E, int bm, int tn,
-                        int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s);
+cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, const int32_t* sorted, int N, int P,
+                        int E, int bm, int tn, int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s);
 
 struct GemmParams {
   int gateup;          // 1: gate/up with SiLU*mul epilogue, 0: down projection
