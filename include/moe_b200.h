@@ -85,7 +85,7 @@ MOE_API const char* moe_last_cuda_error(void);
  * library was built with.  Major 2: moe_topk_gate takes bias_mode and
  * n_shared, moe_forward_args ends with n_shared and bias_mode.  Major 3:
  * moe_ffn_args and moe_forward_args end with the MX weight scales; MX weight
- * types; moe_mx_tile_scales, moe_mx_quantize_rows. */
+ * types; moe_mx_tile_scales, moe_mx_quantize_rows; moe_backward. */
 #define MOE_ABI_VERSION 300
 MOE_API int moe_version(void);
 
@@ -299,6 +299,48 @@ typedef struct {
 MOE_API moe_status_t moe_forward_workspace(const moe_forward_args* args, size_t* ws_bytes);
 MOE_API moe_status_t moe_forward(const moe_forward_args* args, void* ws, size_t ws_bytes,
                          int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_backward -- gradients of the layer forward (bf16 weights).
+ * Passage: MoE Align & Sort article, "Megatron" (the combine's gradient is the
+ * unpermute of the output gradient) and the opening definition of the layer;
+ * the pages print no backward formulas, these are the chain rule through
+ * moe_forward's arithmetic.  With L = sum(out * dout):
+ *   dx       f32 [T, H]          dL/dx
+ *   dlogits  f32 [T, E]          dL/dlogits: the renormalised top-k softmax's
+ *                                gradient at the chosen experts, 0 elsewhere
+ *                                (the choice itself is piecewise constant)
+ *   dw13     f32 [E+S, 2I, H]    dL/dW13 (gate rows, then up rows); zero for
+ *                                experts that no token reached
+ *   dw2      f32 [E+S, H, I]     dL/dW2
+ * Conventions as the forward's reference: the bf16 rounding of h passes the
+ * gradient through unchanged (dh is the gradient of silu(g) * u, dW2 uses
+ * the rounded h); shared experts' weight 1 is a constant.  Routing is
+ * recomputed from the logits (the same arithmetic as moe_topk_gate and
+ * moe_align_sort), and so is the gate/up projection (activations are not
+ * kept by the forward).  Intermediate operands of the gradient GEMMs are bf16
+ * (dout, [dg; du], w * h), accumulation fp32.  All outputs are overwritten.
+ * Limits: as moe_forward with bf16 weights, and block_size % 16 == 0
+ * (MOE_ERR_UNSUPPORTED otherwise).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int T, H, I, E, k, block_size;
+  int n_shared;               /* shared experts after the E routed ones       */
+  int bias_mode;              /* MOE_BIAS_LOGITS or MOE_BIAS_SELECT           */
+  const void* x;              /* bf16 [T, H]                                  */
+  const float* logits;        /* f32 [T, E]                                   */
+  const float* bias;          /* f32 [E], nullable                            */
+  const void* w13;            /* bf16 [E + n_shared, 2I, H]                   */
+  const void* w2;             /* bf16 [E + n_shared, H, I]                    */
+  const void* dout;           /* bf16 [T, H] gradient of the layer output      */
+  float* dx;                  /* out [T, H]                                   */
+  float* dlogits;             /* out [T, E]                                   */
+  float* dw13;                /* out [E + n_shared, 2I, H]                    */
+  float* dw2;                 /* out [E + n_shared, H, I]                     */
+} moe_backward_args;
+MOE_API moe_status_t moe_backward_workspace(const moe_backward_args* args, size_t* ws_bytes);
+MOE_API moe_status_t moe_backward(const moe_backward_args* args, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                  void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_mx_tile_scales -- lay out MX weight scales for the block-scaled GEMM.

@@ -26,6 +26,7 @@ EXPORTED = [
     "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
     "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
     "moe_align_sort_noalloc", "moe_test_quant_division", "moe_mx_tile_scales", "moe_mx_quantize_rows",
+    "moe_backward_workspace", "moe_backward",
 ]
 
 _vp = ctypes.c_void_p
@@ -45,6 +46,12 @@ class ForwardArgs(ctypes.Structure):
                 ("w13", _vp), ("w13_scale", _vp), ("w2", _vp), ("w2_scale", _vp), ("out", _vp),
                 ("topk_ids", _vp), ("topk_w", _vp), ("tile_tokens", _i), ("stage_events", _vp),
                 ("n_shared", _i), ("bias_mode", _i), ("w13_mx_scale", _vp), ("w2_mx_scale", _vp)]
+
+
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("T", _i), ("H", _i), ("I", _i), ("E", _i), ("k", _i), ("block_size", _i), ("n_shared", _i),
+                ("bias_mode", _i), ("x", _vp), ("logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
+                ("dout", _vp), ("dx", _vp), ("dlogits", _vp), ("dw13", _vp), ("dw2", _vp)]
 
 
 MOE_BIAS_LOGITS, MOE_BIAS_SELECT = 0, 1
@@ -81,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_test_quant_division": (_i, [_vp, _vp]),
             "moe_mx_tile_scales": (_i, [_vp, ctypes.c_longlong, _i, _vp, _vp]),
             "moe_mx_quantize_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+            "moe_backward_workspace": (_i, [ctypes.POINTER(BackwardArgs), sz]),
+            "moe_backward": (_i, [ctypes.POINTER(BackwardArgs), _vp, ctypes.c_size_t, _vp, _vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -304,6 +313,34 @@ class MoELayer:
         _check(lib.moe_forward(ctypes.byref(a), _ptr(self._ws), self._ws.numel(),
                                _dev_status(dev_status, x.device), _stream(x.device)), "moe_forward")
         return out
+
+
+def backward(x, logits, w13, w2, dout, k, block_size, bias=None, bias_mode="logits", n_shared=0,
+             dev_status=None, ws=None):
+    """Gradients of sum(out * dout) for the layer forward (bf16 weights):
+    returns (dx f32 [T, H], dlogits f32 [T, E], dw13 f32 like w13, dw2 f32
+    like w2)."""
+    lib = load_library()
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w13.shape[1] // 2
+    dev = x.device
+    dx = torch.empty(T, H, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dw13 = torch.empty(w13.shape, dtype=torch.float32, device=dev)
+    dw2 = torch.empty(w2.shape, dtype=torch.float32, device=dev)
+    a = BackwardArgs(T=T, H=H, I=I, E=E, k=k, block_size=block_size, n_shared=n_shared,
+                     bias_mode=_BIAS_MODES[bias_mode], x=x.data_ptr(), logits=logits.data_ptr(),
+                     bias=None if bias is None else bias.data_ptr(), w13=w13.data_ptr(), w2=w2.data_ptr(),
+                     dout=dout.data_ptr(), dx=dx.data_ptr(), dlogits=dl.data_ptr(), dw13=dw13.data_ptr(),
+                     dw2=dw2.data_ptr())
+    n = ctypes.c_size_t()
+    _check(lib.moe_backward_workspace(ctypes.byref(a), ctypes.byref(n)), "moe_backward_workspace")
+    if ws is None or ws.numel() < n.value:
+        ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
+    _check(lib.moe_backward(ctypes.byref(a), _ptr(ws), ws.numel(), _dev_status(dev_status, dev), _stream(dev)),
+           "moe_backward")
+    return dx, dl, dw13, dw2
 
 
 def mx_tile_scales(sf: torch.Tensor) -> torch.Tensor:

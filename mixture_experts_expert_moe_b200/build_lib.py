@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
-SOURCES = ["api.cu", "align_sort.cu", "elementwise.cu", "grouped_gemm.cu", "mx.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "align_sort.cu", "bwd.cu", "elementwise.cu", "grouped_gemm.cu", "mx.cu", "noalloc.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

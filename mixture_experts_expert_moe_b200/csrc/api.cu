@@ -590,6 +590,173 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// backward
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+struct BwdWs {
+  size_t ids, w, sorted, eids, npost, align, plan, X, D, Z, hw, dgu, dwt, total;
+};
+
+moe_status_t bwd_shape(const moe_backward_args* a, FfnShape* s) {
+  if (a->bias_mode != MOE_BIAS_LOGITS && a->bias_mode != MOE_BIAS_SELECT) return MOE_ERR_INVALID_ARG;
+  if (a->n_shared < 0 || a->E < 1 || a->k < 1 || a->k > a->E || a->k + a->n_shared > 32 ||
+      a->E + a->n_shared > 1024)
+    return MOE_ERR_INVALID_ARG;
+  moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E + a->n_shared, a->k + a->n_shared, a->block_size, MOE_BF16,
+                              0, s);
+  if (st) return st;
+  // the weight gradients multiply whole 16-row MMA steps of an expert's segment
+  if (a->block_size % 16) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+BwdWs bwd_ws_layout(const FfnShape& s) {
+  Carver c;
+  BwdWs w;
+  w.ids = c.take((size_t)s.N * 4);
+  w.w = c.take((size_t)s.N * 4);
+  w.sorted = c.take((size_t)s.P * 4);
+  w.eids = c.take((size_t)s.NB * 4);
+  w.npost = c.take(4);
+  w.align = c.take(align_ws_bytes(s.E));
+  w.plan = c.take((size_t)moe::plan_ints(s.E) * 4);
+  w.X = c.take((size_t)s.P * s.H * 2);     // x rows in sorted order (bf16; padding rows zero)
+  w.D = c.take((size_t)s.P * s.H * 2);     // dout rows in sorted order
+  w.Z = c.take((size_t)s.P * s.I * 4);     // z = D . Wd (fp32)
+  w.hw = c.take((size_t)s.P * s.I * 2);    // w * h (bf16)
+  w.dgu = c.take((size_t)s.P * s.I * 4);   // [dg; du] (bf16, 2I per row)
+  w.dwt = c.take((size_t)s.N * 4);         // combine-weight gradient per slot
+  w.total = c.off;
+  return w;
+}
+
+moe_status_t bwd_fail(int r, const char* what) {
+  if (r == -1) {
+    g_last_cuda_error = std::string(what) + ": cuTensorMapEncodeTiled failed";
+    return MOE_ERR_CUDA;
+  }
+  return cuda_fail((cudaError_t)r, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_backward_workspace(const moe_backward_args* a, size_t* ws_bytes) {
+  if (!a || !ws_bytes) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = bwd_shape(a, &s);
+  if (st) return st;
+  *ws_bytes = bwd_ws_layout(s).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_backward(const moe_backward_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
+                          void* stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  FfnShape s;
+  moe_status_t st = bwd_shape(a, &s);
+  if (st) return st;
+  if (!a->w13 || !a->w2 || !a->dw13 || !a->dw2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->w13) || !aligned16(a->w2) || !aligned16(a->dw13) || !aligned16(a->dw2))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t cs = (cudaStream_t)stream;
+  const size_t EW = (size_t)s.E;
+  if (s.T == 0) {
+    st = check_device();
+    if (st) return st;
+    MOE_CU(cudaMemsetAsync(a->dw13, 0, EW * 2 * s.I * s.H * 4, cs));
+    MOE_CU(cudaMemsetAsync(a->dw2, 0, EW * s.H * s.I * 4, cs));
+    return MOE_OK;
+  }
+  if (!a->x || !a->logits || !a->dout || !a->dx || !a->dlogits || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->x) || !aligned16(a->dout) || !aligned16(a->dx) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  const BwdWs L = bwd_ws_layout(s);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* ids = reinterpret_cast<int32_t*>(w + L.ids);
+  float* tw = reinterpret_cast<float*>(w + L.w);
+  int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
+  int32_t* eids = reinterpret_cast<int32_t*>(w + L.eids);
+  int32_t* npost = reinterpret_cast<int32_t*>(w + L.npost);
+  int32_t* plan = reinterpret_cast<int32_t*>(w + L.plan);
+  void* X = w + L.X;
+  void* D = w + L.D;
+  float* Z = reinterpret_cast<float*>(w + L.Z);
+  __nv_bfloat16* hw = reinterpret_cast<__nv_bfloat16*>(w + L.hw);
+  __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(w + L.dgu);
+  float* dwt = reinterpret_cast<float*>(w + L.dwt);
+  const int N = (int)s.N, R = (int)s.rows_max;
+  const int ks = s.k, kr = a->k;   // slots per token, routed choices
+
+  // routing (gate + align & sort + tile plan), then the token rows in sorted order
+  st = run_route(s, a->n_shared, a->bias_mode == MOE_BIAS_SELECT, a->logits, a->bias, ids, tw, sorted, eids, npost,
+                 w + L.align, plan, dev_status, cs);
+  if (st) return st;
+  MOE_CU(moe::launch_gather_rows(a->x, nullptr, sorted, npost, R, N, ks, s.H * 2, X, nullptr, cs));
+  MOE_CU(moe::launch_gather_rows(a->dout, nullptr, sorted, npost, R, N, ks, s.H * 2, D, nullptr, cs));
+
+  moe::BwdLaunch g = {};
+  g.p.E = s.E;
+  g.p.k = ks;
+  g.p.n_slots = N;
+  g.p.plan = plan;
+  g.p.sorted = sorted;
+  g.p.status = dev_status;
+  g.p.timeout_ns = moe::kDefaultTimeoutNs;
+  g.p.tn = s.tn;
+  // z = D . Wd (Wd read transposed)
+  moe::BwdLaunch gz = g;
+  gz.a = a->w2; gz.a_rows = (long long)EW * s.H; gz.a_cols = s.I;
+  gz.b = D; gz.b_rows = s.P; gz.b_cols = s.H;
+  gz.p.kind = moe::BWD_Z; gz.p.K = s.H; gz.p.n_out = s.I; gz.p.out = Z;
+  int r = moe::launch_bwd_gemm(gz, cs);
+  if (r) return bwd_fail(r, "backward z GEMM");
+  // gate/up recomputed with the SwiGLU backward in the epilogue (padding rows of hw / dgu stay zero)
+  MOE_CU(cudaMemsetAsync(hw, 0, (size_t)s.P * s.I * 2, cs));
+  MOE_CU(cudaMemsetAsync(dgu, 0, (size_t)s.P * s.I * 4, cs));
+  MOE_CU(cudaMemsetAsync(dwt, 0, (size_t)N * 4, cs));
+  moe::BwdLaunch gg = g;
+  gg.a = a->w13; gg.a_rows = (long long)EW * 2 * s.I; gg.a_cols = s.H;
+  gg.b = X; gg.b_rows = s.P; gg.b_cols = s.H;
+  gg.p.kind = moe::BWD_GUB; gg.p.K = s.H; gg.p.n_out = s.I;
+  gg.p.topk_w = tw; gg.p.zbuf = Z; gg.p.hw = hw; gg.p.dgu = dgu; gg.p.dwt = dwt;
+  r = moe::launch_bwd_gemm(gg, cs);
+  if (r) return bwd_fail(r, "backward gate/up GEMM");
+  // dx: per slot dgu . W13 (W13 read transposed), added into the token's row
+  MOE_CU(cudaMemsetAsync(a->dx, 0, (size_t)s.T * s.H * 4, cs));
+  moe::BwdLaunch gx = g;
+  gx.a = a->w13; gx.a_rows = (long long)EW * 2 * s.I; gx.a_cols = s.H;
+  gx.b = dgu; gx.b_rows = s.P; gx.b_cols = 2 * s.I;
+  gx.p.kind = moe::BWD_DX; gx.p.K = 2 * s.I; gx.p.n_out = s.H; gx.p.dx = a->dx;
+  r = moe::launch_bwd_gemm(gx, cs);
+  if (r) return bwd_fail(r, "backward dx GEMM");
+  // router logits
+  MOE_CU(moe::launch_dlogits(ids, tw, dwt, s.T, a->E, kr, ks, a->dlogits, cs));
+  // weight gradients, per expert over its sorted rows
+  moe::BwdLaunch g2 = g;
+  g2.a = D; g2.a_rows = s.P; g2.a_cols = s.H;
+  g2.b = hw; g2.b_rows = s.P; g2.b_cols = s.I;
+  g2.p.kind = moe::BWD_WG; g2.p.n_out = s.H; g2.p.n_cols = s.I; g2.p.out = a->dw2;
+  g2.p.tn = s.I % 256 == 0 ? 256 : 128;
+  r = moe::launch_bwd_gemm(g2, cs);
+  if (r) return bwd_fail(r, "backward dW2 GEMM");
+  moe::BwdLaunch g13 = g;
+  g13.a = dgu; g13.a_rows = s.P; g13.a_cols = 2 * s.I;
+  g13.b = X; g13.b_rows = s.P; g13.b_cols = s.H;
+  g13.p.kind = moe::BWD_WG; g13.p.n_out = 2 * s.I; g13.p.n_cols = s.H; g13.p.out = a->dw13;
+  g13.p.tn = s.H % 256 == 0 ? 256 : 128;
+  r = moe::launch_bwd_gemm(g13, cs);
+  if (r) return bwd_fail(r, "backward dW13 GEMM");
+  return MOE_OK;
+}
+
 moe_status_t moe_mx_tile_scales(const uint8_t* sf, long long rows, int K, uint8_t* out, void* stream) {
   if (rows < 0 || K < 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
   if (rows == 0 || K == 0) return MOE_OK;

@@ -261,6 +261,30 @@ __host__ __device__ __forceinline__ uint32_t umma_idesc_mx(int M, int N, uint32_
          ((uint32_t)(M >> 4) << 24) | (sf_id << 29);
 }
 
+// Shared-memory descriptor of an MN-major operand tile with 128-byte swizzle,
+// as TMA writes it from boxes of 64 bf16 along M (or N) by K rows: box c
+// (elements 64c..64c+63 along M/N) at offset c * box_bytes, K-row k of a box
+// at k * 128 bytes (swizzle atoms of 8 K-rows = 1024 bytes).  The leading
+// byte offset steps to the next 64 elements along M/N, the stride byte offset
+// to the next 8 K-rows; one MMA K-step of 16 rows advances the start address
+// by 2048 bytes.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t smem_addr, uint32_t box_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)((box_bytes >> 4) & 0x3FFF) << 16;  // leading byte offset: next 64 M/N elements
+  d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: next 8 K-rows
+  d |= (uint64_t)1 << 46;                             // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                             // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with operand majors: a_mn / b_mn = 1 for
+// an MN-major A / B (0 = K-major), bf16 operands, fp32 accumulator.
+__host__ __device__ __forceinline__ uint32_t umma_idesc_bf16_major(int M, int N, uint32_t a_mn, uint32_t b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor: fp32 accumulator, A/B K-major, shape M x N.
 // fmt: 1 = bf16 (kind::f16), 0 = E4M3 (kind::f8f6f4).
 __host__ __device__ __forceinline__ uint32_t umma_idesc(int M, int N, uint32_t fmt) {

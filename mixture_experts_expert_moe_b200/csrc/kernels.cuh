@@ -137,6 +137,45 @@ struct GemmLaunch {
   GemmParams p;
 };
 
+// Backward GEMMs (bwd.cu): the tile kinds and their operands.
+enum BwdKind {
+  BWD_Z = 0,     // z [P, I] = D_r . Wd[e] (transposed weights): fp32 rows
+  BWD_GUB = 1,   // gate/up recomputed; epilogue: SwiGLU backward -> dgu, w*h, combine-weight gradient
+  BWD_DX = 2,    // dx [T, H] += dgu_r . W13[e] (transposed weights), fp32 additions per token
+  BWD_WG = 3     // weight gradient of one expert: [M, N] = A^T B over its sorted token rows (fp32)
+};
+struct BwdParams {
+  int kind;
+  int K;              // reduction length (Z: H; GUB: H; DX: 2I; WG: the expert's rows)
+  int n_out;          // M: output features (Z, GUB: I; DX: H) or rows of the weight gradient
+  int n_cols;         // WG: columns of the weight gradient
+  int tn;             // token tile (Z, GUB, DX) or column tile (WG, 128 or 256)
+  int stages, n_acc, tmem_cols;
+  int E, k, n_slots;
+  const int32_t* plan;
+  const int32_t* sorted;
+  const float* topk_w;   // GUB: routing weights per slot
+  const float* zbuf;     // GUB: z [P, I]
+  float* out;            // Z: z [P, I]; WG: dW [E, n_out, n_cols]
+  __nv_bfloat16* hw;     // GUB: w * h [P, I]
+  __nv_bfloat16* dgu;    // GUB: [dg; du] [P, 2I]
+  float* dwt;            // GUB: gradient of each slot's combine weight (atomic sums)
+  float* dx;             // DX: [T, n_out] fp32
+  int32_t* status;
+  long long timeout_ns;
+};
+struct BwdLaunch {
+  const void* a;             // A source [a_rows, a_cols] bf16 (K-major weights, or MN-major)
+  long long a_rows, a_cols;
+  const void* b;             // B source [b_rows, b_cols] bf16
+  long long b_rows, b_cols;
+  BwdParams p;
+};
+// returns 0 on success, -1 if a tensor map could not be encoded, else a cudaError_t
+int launch_bwd_gemm(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_dlogits(const int32_t* ids, const float* w, const float* dwt, int T, int E, int k, int kk,
+                           float* dlogits, cudaStream_t s);
+
 size_t gemm_smem_bytes(int tn, int stages, int E, bool mx);
 int gemm_pick_stages(int tn, int E, bool mx);
 // returns 0 on success, -1 if a tensor map could not be encoded, else a cudaError_t
