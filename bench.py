@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 from moe_inputs import ALIGN_CONFIG, CONFIGS, align_ids, make_layer, pack_e2m1  # noqa: E402
 from mixture_experts_expert_moe_b200.roofline import (  # noqa: E402
-    align_bytes, down_kernel_bytes, gateup_kernel_bytes, layer_bytes, moe_flops)
+    align_bytes, backward_bytes, backward_flops, down_kernel_bytes, gateup_kernel_bytes, layer_bytes, moe_flops)
 
 METRIC = "MoE layer tokens/s & TFLOPS vs roofline (bf16/fp8); align&sort µs, GB/s"
 PRIMARY = CONFIGS["deepseek"]
@@ -351,6 +351,50 @@ def layer_report(m, cfg, steps, warmup, dev, pk, dtype_name, primary=False, tile
     return rep, e2e, ms
 
 
+def backward_report(m, cfg, steps, warmup, dev, pk):
+    """One moe_backward (gradients of x, the router logits and both weight
+    tensors; bf16 weights) on the layer, timed with CUDA events."""
+    from moe_inputs import normal
+    d = make_layer(cfg, device=dev)
+    dout = normal((cfg.T, cfg.H), 1.0, cfg.seed * 16 + 9, dev, torch.bfloat16)
+    outs = (torch.empty(cfg.T, cfg.H, dtype=torch.float32, device=dev),
+            torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev),
+            torch.empty(d["w13"].shape, dtype=torch.float32, device=dev),
+            torch.empty(d["w2"].shape, dtype=torch.float32, device=dev))
+    ws = None
+
+    def call():
+        m.backward(d["x"], d["logits"], d["w13"], d["w2"], dout, cfg.k, cfg.bm, bias=d["bias"],
+                   bias_mode=cfg.bias_mode, n_shared=cfg.n_shared, outs=outs, ws=ws)
+
+    call()
+    torch.cuda.synchronize()
+    ids = torch.topk(d["logits"], cfg.k, dim=1).indices
+    touched = int(torch.unique(ids).numel()) + cfg.n_shared
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        call()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    pairs = slot_pairs(cfg)
+    fl = backward_flops(pairs, cfg.H, cfg.I)
+    by = backward_bytes(cfg.T, cfg.H, cfg.I, cfg.E + cfg.n_shared, touched, cfg.E)
+    t_roof = max(fl / (pk["bf16_tflops_sustained"] * 1e12), by / (pk["hbm_gbs"] * 1e9)) * 1e3
+    del d, dout, outs
+    torch.cuda.empty_cache()
+    return {"workload": "backward " + workload_name(cfg, "bf16"), "ms_per_step": ms,
+            "tokens_per_s": cfg.T / (ms * 1e-3), "tflops": fl / (ms * 1e-3) / 1e12, "touched_experts": touched,
+            "roofline_ms": t_roof, "roofline_frac": t_roof / ms,
+            "bound": "tensor" if fl / (pk["bf16_tflops_sustained"] * 1e12) > by / (pk["hbm_gbs"] * 1e9) else "hbm",
+            "algorithmic_bytes": by, "flops": fl,
+            "note": "dW13/dW2 in fp32 for all experts; gate/up recomputed; eager launches"}
+
+
 def bm_sweep(m, cfg, steps, warmup, dev, pk, sizes=(32, 64, 128)):
     """The layer at several block sizes (routing and values unchanged; the
     padding and the GEMM token groups change), in bf16 and a8w8, each
@@ -504,6 +548,7 @@ def run_ours(args):
                 extra["decode_mx"].append(layer_report(m, c, 100, 5, dev, pk, fmt)[0])
         extra["deepseek_mx"] = [layer_report(m, cfg.with_(mx=fmt), 30, 3, dev, pk, fmt)[0]
                                 for fmt in ("mxfp4", "mxfp8")]
+        extra["backward"] = backward_report(m, cfg, 10, 3, dev, pk)
         extra["align_sort"] = align_report(m, dev, pk, ALIGN_CONFIG["T"])
         extra["align_sort_large"] = align_report(m, dev, pk, 1 << 22, iters=20)
     cpu = None
@@ -705,6 +750,15 @@ def run_only(args):
     steps = 20 if args.steps is None else args.steps
     warmup = 3 if args.warmup is None else max(3, args.warmup)
     parts = args.only.split("_")
+    if parts[0] == "backward":      # backward_<config>[_T<N>][_E<N>]
+        cfg = CONFIGS[parts[1]]
+        for q in parts[2:]:
+            if q.startswith("T"):
+                cfg = cfg.with_(T=int(q[1:]))
+            elif q.startswith("E"):
+                cfg = cfg.with_(E=int(q[1:]))
+        print(json.dumps(backward_report(m, cfg, steps, warmup, dev, pk)))
+        return
     if parts[0] == "align":
         print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
         return

@@ -316,19 +316,21 @@ class MoELayer:
 
 
 def backward(x, logits, w13, w2, dout, k, block_size, bias=None, bias_mode="logits", n_shared=0,
-             dev_status=None, ws=None):
+             dev_status=None, ws=None, outs=None):
     """Gradients of sum(out * dout) for the layer forward (bf16 weights):
     returns (dx f32 [T, H], dlogits f32 [T, E], dw13 f32 like w13, dw2 f32
-    like w2)."""
+    like w2), written into ``outs`` when given."""
     lib = load_library()
     T, H = x.shape
     E = logits.shape[1]
     I = w13.shape[1] // 2
     dev = x.device
-    dx = torch.empty(T, H, dtype=torch.float32, device=dev)
-    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
-    dw13 = torch.empty(w13.shape, dtype=torch.float32, device=dev)
-    dw2 = torch.empty(w2.shape, dtype=torch.float32, device=dev)
+    if outs is None:
+        outs = (torch.empty(T, H, dtype=torch.float32, device=dev),
+                torch.empty(T, E, dtype=torch.float32, device=dev),
+                torch.empty(w13.shape, dtype=torch.float32, device=dev),
+                torch.empty(w2.shape, dtype=torch.float32, device=dev))
+    dx, dl, dw13, dw2 = outs
     a = BackwardArgs(T=T, H=H, I=I, E=E, k=k, block_size=block_size, n_shared=n_shared,
                      bias_mode=_BIAS_MODES[bias_mode], x=x.data_ptr(), logits=logits.data_ptr(),
                      bias=None if bias is None else bias.data_ptr(), w13=w13.data_ptr(), w2=w2.data_ptr(),

@@ -70,3 +70,19 @@ def down_kernel_bytes(T: int, H: int, I: int, touched: int, pairs: int, a8w8: bo
     routing it reads (slot id and weight per pair).  The h operand and
     padding are not counted."""
     return touched * _weight_matrix_bytes(H, I, a8w8, mx) + T * H * 4 + pairs * 8
+
+
+def backward_flops(pairs: int, H: int, I: int) -> float:
+    """FLOPs of the expert FFN's backward with the gate/up projection
+    recomputed: z = Wd^T dout (2 pairs H I), gate/up again (4), dx (4), dW2
+    (2) and dW13 (4) -> 16 pairs H I."""
+    return 16.0 * pairs * H * I
+
+
+def backward_bytes(T: int, H: int, I: int, E_all: int, touched: int, E_logits: int) -> int:
+    """Algorithmic bytes of moe_backward (bf16 weights): the touched experts'
+    gate/up weights read twice (recomputation, dx) and down weights once; the
+    fp32 weight gradients of every expert written once; x and dout read once
+    (bf16), dx written once (fp32), logits read and their gradient written."""
+    return (touched * (2 * (2 * I * H * 2) + H * I * 2) + E_all * 3 * H * I * 4
+            + 2 * T * H * 2 + T * H * 4 + 2 * T * E_logits * 4)

@@ -81,3 +81,14 @@ def test_mx_weight_bytes_by_hand():
     cfg = MoEConfig("t", T=4, H=H, I=I, E=8, k=2, bm=16, mx="mxfp4")
     assert bench.gateup_bytes(cfg, 3) == 3 * (2 * I * H // 2 + 2 * I * H // 32) + 4 * H + 8 * 4
     assert bench.down_bytes(cfg, 3) == 3 * (H * I // 2 + H * I // 32) + 4 * H * 4 + 8 * 8
+
+
+def test_backward_accounting_by_hand():
+    from mixture_experts_expert_moe_b200.roofline import backward_bytes, backward_flops
+    # z (2) + gate/up again (4) + dx (4) + dW2 (2) + dW13 (4) multiply-add FLOPs per pair, H, I
+    assert backward_flops(10, 256, 128) == 16 * 10 * 256 * 128
+    T, H, I, E, touched, EL = 4, 256, 128, 8, 3, 8
+    w_read = touched * (2 * 2 * I * H * 2 + H * I * 2)       # W13 twice, Wd once (bf16)
+    dw = E * 3 * H * I * 4                                     # fp32 gradients of every expert
+    act = 2 * T * H * 2 + T * H * 4 + 2 * T * EL * 4           # x, dout in; dx out; logits in, dlogits out
+    assert backward_bytes(T, H, I, E, touched, EL) == w_read + dw + act

@@ -103,7 +103,8 @@ def test_mx_forward_parity(cuda_device, name, cfg, smean, n_sample, elem):
                                          w_elem=elem, bias=to_numpy(d["bias"]), tokens=toks)
     np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
     got = out[torch.from_numpy(toks).to(cuda_device)].cpu().numpy()
-    assert_close(got, ref, TOL_FP8, f"{name} {mx}")
+    err = assert_close(got, ref, TOL_FP8, f"{name} {mx}")
+    print(f"{name} {mx}: max abs {err[0]:.2e}, rel fro {err[1]:.2e}, max |ref| {np.abs(ref).max():.2e}")
 
 
 @pytest.mark.parametrize("elem", ["e2m1", "e4m3"])
