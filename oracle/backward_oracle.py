@@ -40,12 +40,18 @@ def _sigmoid(g):
     return 1.0 / (1.0 + np.exp(-g))
 
 
-def moe_backward(x, logits, k, w13, w2, dout, bias=None, bias_mode="logits", n_shared=0):
+def moe_backward(x, logits, k, w13, w2, dout, bias=None, bias_mode="logits", n_shared=0, tokens=None,
+                 experts=None):
     """Gradients of sum(out * dout) for the layer of ``moe_forward``.
 
     x [T, H], logits [T, E] (E routed experts), w13 [E+S, 2I, H],
     w2 [E+S, H, I], dout [T, H].  Returns (dx [T, H], dlogits [T, E],
     dw13 [E+S, 2I, H], dw2 [E+S, H, I]) in float64.
+
+    ``tokens`` / ``experts`` (for large layers) restrict the work: dx and
+    dlogits are computed for the listed tokens only and the weight gradients
+    for the listed experts only (the other entries are left zero); each
+    computed entry is the same sum as without the restriction.
     """
     x = np.asarray(x, dtype=np.float64)
     dout = np.asarray(dout, dtype=np.float64)
@@ -64,9 +70,15 @@ def moe_backward(x, logits, k, w13, w2, dout, bias=None, bias_mode="logits", n_s
     dw2 = np.zeros((EW, H, I))
     dwt = np.zeros((T, kk))            # d loss / d w[t, j]
 
+    want_t = np.ones(T, dtype=bool) if tokens is None else np.isin(np.arange(T), np.asarray(tokens))
+    want_e = None if experts is None else set(int(e) for e in experts)
     for t in range(T):
         for j in range(kk):
             e = int(ids[t, j])
+            for_t = bool(want_t[t])
+            for_e = want_e is None or e in want_e
+            if not (for_t or for_e):
+                continue
             W13 = np.asarray(w13[e], dtype=np.float64)
             Wd = np.asarray(w2[e], dtype=np.float64)
             # forward of this slot, as the oracle computes it
@@ -79,7 +91,8 @@ def moe_backward(x, logits, k, w13, w2, dout, bias=None, bias_mode="logits", n_s
             dwt[t, j] = dout[t] @ y
             dy = w[t, j] * dout[t]
             # down projection
-            dw2[e] += np.outer(dy, h)
+            if for_e:
+                dw2[e] += np.outer(dy, h)
             dh = Wd.T @ dy                 # straight through the bf16 rounding
             # SwiGLU
             du = dh * a
@@ -88,12 +101,14 @@ def moe_backward(x, logits, k, w13, w2, dout, bias=None, bias_mode="logits", n_s
             dg = da * (s * (1.0 + g * (1.0 - s)))
             # gate/up projection
             dgu = np.concatenate([dg, du])
-            dw13[e] += np.outer(dgu, x[t])
-            dx[t] += W13.T @ dgu
+            if for_e:
+                dw13[e] += np.outer(dgu, x[t])
+            if for_t:
+                dx[t] += W13.T @ dgu
 
     # renormalised softmax over the k routed choices (shared columns have w = 1)
     dlogits = np.zeros((T, E))
-    for t in range(T):
+    for t in np.nonzero(want_t)[0]:
         wr = w[t, :k]
         g_w = dwt[t, :k]
         dl_sel = wr * (g_w - np.dot(wr, g_w))

@@ -100,3 +100,19 @@ def test_backward_finite_differences_logits_and_down_weights():
     for t in range(4):
         mask[t, ids[t]] = False
     assert np.all(dl[mask] == 0)
+
+
+def test_restricted_backward_equals_the_full_one():
+    """Restricting the oracle to some tokens and experts leaves the computed
+    entries unchanged and the others zero."""
+    x, logits, w13, w2, dout, bias = _layer(T=12, H=16, I=8, E=5, k=2, S=1, seed=4)
+    full = bo.moe_backward(x, logits, 2, w13, w2, dout, bias=bias, bias_mode="select", n_shared=1)
+    toks, exps = [1, 7], [0, 5]
+    part = bo.moe_backward(x, logits, 2, w13, w2, dout, bias=bias, bias_mode="select", n_shared=1,
+                           tokens=toks, experts=exps)
+    for a, b in zip(full[:2], part[:2]):
+        np.testing.assert_array_equal(b[toks], a[toks])
+        assert not np.any(np.delete(b, toks, axis=0))
+    for a, b in zip(full[2:], part[2:]):
+        np.testing.assert_array_equal(b[exps], a[exps])
+        assert not np.any(np.delete(b, exps, axis=0))
