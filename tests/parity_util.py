@@ -27,6 +27,16 @@ def assert_close(got, ref, tol, what=""):
     return max_abs, rel
 
 
+def assert_close_scaled(got, ref, tol, what=""):
+    """assert_close with the max-abs bar taken relative to the output's scale:
+    |got - ref| <= tol[0] * max(1, max |ref|) (the relative Frobenius bar is
+    unchanged).  For gradients summed over many tokens, whose entries grow with
+    the sum while their bf16 operands keep 8 significant bits, an absolute bar
+    meant for outputs of order 1 would be tighter than one bf16 ulp."""
+    scale = max(1.0, float(np.max(np.abs(np.asarray(ref, dtype=np.float64)))) if np.size(ref) else 1.0)
+    return assert_close(got, ref, (tol[0] * scale, tol[1]), what)
+
+
 def bf16_ulp(v):
     """Spacing of bfloat16 values at |v| (normal range)."""
     a = np.maximum(np.abs(np.asarray(v, dtype=np.float64)), 2.0 ** -126)

@@ -36,3 +36,15 @@ def test_pack_e2m1_layout_numpy_and_torch():
     assert tc.dtype == torch.uint8 and ts.shape == (2, 4, 2)
     assert not bool(((tc & 0x7F) == 0x7F).any())        # no NaN codes
     assert int(ts.min()) >= 121 and int(ts.max()) <= 123
+
+
+def test_scaled_tolerance_follows_the_output_scale():
+    import pytest
+    from parity_util import assert_close_scaled
+    ref = np.array([100.0, -50.0, 1.0])
+    assert_close_scaled(ref + 1.5, ref, (2e-2, 1.0))           # 1.5 <= 2e-2 * 100
+    with pytest.raises(AssertionError):
+        assert_close_scaled(ref + 2.5, ref, (2e-2, 1.0))
+    small = np.array([0.5, -0.25])
+    with pytest.raises(AssertionError):
+        assert_close_scaled(small + 0.03, small, (2e-2, 1.0))  # scale floor 1: bar stays 2e-2
