@@ -119,3 +119,37 @@ def test_mx_grouped_ffn_parity(cuda_device, elem):
     torch.cuda.synchronize()
     ref = mxo.ffn_mx(to_numpy(d["x"]), ids.cpu().numpy(), w13c, w13s, w2c, w2s, w_elem=elem)
     assert_close(y.cpu().numpy(), ref, TOL_FP8, f"grouped ffn {elem}")
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "mxfp8"])
+def test_mx_fullsize_prefill_sampled(cuda_device, fmt):
+    """The DeepSeek-V3-shaped prefill layer with MX weights, in the launch
+    configuration bench.py times (make_layer's MX weights, bf16 output):
+    routing bit-exact, every output finite, and sampled tokens (first, last,
+    the last slot of the most loaded expert, random ones) within the FP8
+    tolerance of the MX oracle."""
+    cfg = CONFIGS["deepseek"].with_(mx=fmt)
+    d = make_layer(cfg, device=cuda_device)
+    pack = pack_e2m1 if fmt == "mxfp4" else (lambda c: c)
+    layer = m.MoELayer(pack(d["w13_codes"]), pack(d["w2_codes"]), cfg.k, cfg.bm, out_dtype=torch.float32, mx=fmt,
+                       w13_mx_scale=m.mx_tile_scales(d["w13_sf"]), w2_mx_scale=m.mx_tile_scales(d["w2_sf"]))
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = layer(d["x"], d["logits"], topk_ids=ids, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and torch.isfinite(out).all()
+    logits = to_numpy(d["logits"])
+    r_ids, _ = mxo.topk_gate(logits, cfg.k)
+    flat = r_ids.reshape(-1)
+    hot = np.argmax(np.bincount(flat, minlength=cfg.E))
+    rng = np.random.default_rng(cfg.seed)
+    toks = np.array(sorted({0, cfg.T - 1, int(np.nonzero(flat == hot)[0][-1] // cfg.k),
+                            *rng.choice(cfg.T, size=9, replace=False).tolist()}))
+    elem = "e2m1" if fmt == "mxfp4" else "e4m3"
+    views = [ExpertView(d[k], codes=True) for k in ("w13_codes", "w13_sf", "w2_codes", "w2_sf")]
+    ref, ref_ids, _ = mxo.moe_forward_mx(to_numpy(d["x"]), logits, cfg.k, *views, w_elem=elem, tokens=toks)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    got = out[torch.from_numpy(toks).to(cuda_device)].cpu().numpy()
+    err = assert_close(got, ref, TOL_FP8, f"deepseek {fmt}")
+    print(f"deepseek {fmt}: {len(toks)} tokens, max abs {err[0]:.2e}, rel fro {err[1]:.2e}, "
+          f"max |ref| {np.abs(ref).max():.2e}")
