@@ -85,7 +85,8 @@ MOE_API const char* moe_last_cuda_error(void);
  * library was built with.  Major 2: moe_topk_gate takes bias_mode and
  * n_shared, moe_forward_args ends with n_shared and bias_mode.  Major 3:
  * moe_ffn_args and moe_forward_args end with the MX weight scales; MX weight
- * types; moe_mx_tile_scales, moe_mx_quantize_rows; moe_backward. */
+ * types; moe_mx_tile_scales, moe_mx_quantize_rows; moe_backward; the
+ * expert-parallel steps moe_ep_route, moe_permute_rows, moe_scatter_rows. */
 #define MOE_ABI_VERSION 300
 MOE_API int moe_version(void);
 
@@ -341,6 +342,41 @@ typedef struct {
 MOE_API moe_status_t moe_backward_workspace(const moe_backward_args* args, size_t* ws_bytes);
 MOE_API moe_status_t moe_backward(const moe_backward_args* args, void* ws, size_t ws_bytes, int32_t* dev_status,
                                   void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert parallelism (EP): the layer's experts sharded over R ranks (rank r
+ * holds experts [r*E/R, (r+1)*E/R)), every rank gating its own tokens.
+ * Passage: X-MoE abstract and GC-MoE abstract (expert-parallel dispatch and
+ * combine across GPUs).  These calls are the per-rank steps; the exchange
+ * between ranks (all-to-all of counts, token rows and expert outputs) is the
+ * caller's collective (NCCL through torch.distributed in the Python binding).
+ *
+ * moe_ep_route: destination ranks of the T*k slots.
+ *   topk_ids    i32 [T*k]  global expert of every slot
+ *   order       i32 [T*k]  out: the flat slots grouped by destination rank
+ *                          (ascending rank, ascending slot inside a rank)
+ *   send_counts i32 [R]    out: slots per destination rank
+ *   local_ids   i32 [T*k]  out: order's slots' expert ids local to their rank
+ *                          (expert % (E/R))
+ *   ws          device workspace of moe_ep_route_workspace's size
+ * Limits: 1 <= R <= 1024, E % R == 0.  Out-of-range ids are skipped and
+ * flagged with MOE_DEV_BAD_EXPERT_ID (order then holds fewer real entries).
+ * ------------------------------------------------------------------------- */
+MOE_API moe_status_t moe_ep_route_workspace(int T, int k, int R, size_t* ws_bytes);
+MOE_API moe_status_t moe_ep_route(const int32_t* topk_ids, int T, int k, int E, int R, int32_t* order,
+                                  int32_t* send_counts, int32_t* local_ids, void* ws, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream);
+/* moe_permute_rows: dst row i = src row map[i] / div for i < n (the permute
+ * before the exchange: div = k turns slots into tokens).  moe_scatter_rows:
+ * dst row map[i] = src row i (the un-permute after it).  Rows of row_bytes
+ * bytes (a multiple of 16), 16-byte-aligned buffers; map entries whose row
+ * falls outside [0, src_rows) / [0, dst_rows) move nothing.
+ * Passage: MoE Align & Sort article, "FasterTransformer" (permute) and
+ * "Megatron" (unpermute). */
+MOE_API moe_status_t moe_permute_rows(const void* src, int row_bytes, const int32_t* map, int n, int div,
+                                      int src_rows, void* dst, void* stream);
+MOE_API moe_status_t moe_scatter_rows(const void* src, int row_bytes, const int32_t* map, int n, int dst_rows,
+                                      void* dst, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_mx_tile_scales -- lay out MX weight scales for the block-scaled GEMM.

@@ -26,7 +26,8 @@ EXPORTED = [
     "moe_align_sort_sizes", "moe_align_sort", "moe_ffn_workspace", "moe_grouped_ffn",
     "moe_combine", "moe_forward_workspace", "moe_forward", "moe_test_wait_timeout",
     "moe_align_sort_noalloc", "moe_test_quant_division", "moe_mx_tile_scales", "moe_mx_quantize_rows",
-    "moe_backward_workspace", "moe_backward",
+    "moe_backward_workspace", "moe_backward", "moe_ep_route_workspace", "moe_ep_route", "moe_permute_rows",
+    "moe_scatter_rows",
 ]
 
 _vp = ctypes.c_void_p
@@ -90,6 +91,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "moe_mx_quantize_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
             "moe_backward_workspace": (_i, [ctypes.POINTER(BackwardArgs), sz]),
             "moe_backward": (_i, [ctypes.POINTER(BackwardArgs), _vp, ctypes.c_size_t, _vp, _vp]),
+            "moe_ep_route_workspace": (_i, [_i, _i, _i, sz]),
+            "moe_ep_route": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]),
+            "moe_permute_rows": (_i, [_vp, _i, _vp, _i, _i, _i, _vp, _vp]),
+            "moe_scatter_rows": (_i, [_vp, _i, _vp, _i, _i, _vp, _vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -343,6 +348,49 @@ def backward(x, logits, w13, w2, dout, k, block_size, bias=None, bias_mode="logi
     _check(lib.moe_backward(ctypes.byref(a), _ptr(ws), ws.numel(), _dev_status(dev_status, dev), _stream(dev)),
            "moe_backward")
     return dx, dl, dw13, dw2
+
+
+def ep_route(topk_ids: torch.Tensor, E: int, R: int, dev_status=None):
+    """Destination ranks of the slots for R-way expert parallelism (rank r
+    holds experts [r*E/R, (r+1)*E/R)): returns (order int32 [T*k]: the flat
+    slots grouped by destination rank, send_counts int32 [R], local_ids int32
+    [T*k]: the slots' expert ids local to their rank, in order's order)."""
+    lib = load_library()
+    assert topk_ids.is_cuda and topk_ids.dtype == torch.int32 and topk_ids.is_contiguous()
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    n = ctypes.c_size_t()
+    _check(lib.moe_ep_route_workspace(T, k, R, ctypes.byref(n)), "moe_ep_route_workspace")
+    ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
+    order = torch.empty(T * k, dtype=torch.int32, device=dev)
+    counts = torch.empty(R, dtype=torch.int32, device=dev)
+    local = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _check(lib.moe_ep_route(_ptr(topk_ids), T, k, E, R, _ptr(order), _ptr(counts), _ptr(local), _ptr(ws),
+                            ws.numel(), _dev_status(dev_status, dev), _stream(dev)), "moe_ep_route")
+    return order, counts, local
+
+
+def permute_rows(src: torch.Tensor, index: torch.Tensor, div: int = 1) -> torch.Tensor:
+    """out[i] = src[index[i] // div] (rows of a 2-D tensor)."""
+    lib = load_library()
+    assert src.is_cuda and src.is_contiguous() and index.dtype == torch.int32
+    n = index.numel()
+    out = torch.empty(n, src.shape[1], dtype=src.dtype, device=src.device)
+    rb = src.shape[1] * src.element_size()
+    _check(lib.moe_permute_rows(_ptr(src), rb, _ptr(index), n, div, src.shape[0], _ptr(out), _stream(src.device)),
+           "moe_permute_rows")
+    return out
+
+
+def scatter_rows(src: torch.Tensor, index: torch.Tensor, rows: int) -> torch.Tensor:
+    """out[index[i]] = src[i]; out has `rows` rows (rows no index names are 0)."""
+    lib = load_library()
+    assert src.is_cuda and src.is_contiguous() and index.dtype == torch.int32
+    out = torch.zeros(rows, src.shape[1], dtype=src.dtype, device=src.device)
+    rb = src.shape[1] * src.element_size()
+    _check(lib.moe_scatter_rows(_ptr(src), rb, _ptr(index), index.numel(), rows, _ptr(out), _stream(src.device)),
+           "moe_scatter_rows")
+    return out
 
 
 def mx_tile_scales(sf: torch.Tensor) -> torch.Tensor:

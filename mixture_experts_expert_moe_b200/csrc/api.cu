@@ -757,6 +757,70 @@ moe_status_t moe_backward(const moe_backward_args* a, void* ws, size_t ws_bytes,
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// expert parallelism: routing of slots to ranks, row permutations
+// ---------------------------------------------------------------------------
+static size_t ep_ws_layout(long long N, int R, size_t* dest, size_t* eids, size_t* npost, size_t* align) {
+  Carver c;
+  *dest = c.take((size_t)N * 4);
+  *eids = c.take((size_t)N * 4);
+  *npost = c.take(4);
+  *align = c.take(align_ws_bytes(R));
+  return c.off;
+}
+
+moe_status_t moe_ep_route_workspace(int T, int k, int R, size_t* ws_bytes) {
+  if (!ws_bytes || !align_args_ok(T, k, R, 1)) return MOE_ERR_INVALID_ARG;
+  size_t a, b, c, d;
+  *ws_bytes = ep_ws_layout((long long)T * k, R, &a, &b, &c, &d);
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_route(const int32_t* topk_ids, int T, int k, int E, int R, int32_t* order, int32_t* send_counts,
+                          int32_t* local_ids, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!align_args_ok(T, k, R, 1) || E < R || E % R) return MOE_ERR_INVALID_ARG;
+  if (!send_counts || (T > 0 && (!topk_ids || !order || !local_ids || !ws))) return MOE_ERR_INVALID_ARG;
+  const long long N = (long long)T * k;
+  size_t o_dest, o_eids, o_np, o_al;
+  if (ws_bytes < ep_ws_layout(N, R, &o_dest, &o_eids, &o_np, &o_al) && T > 0) return MOE_ERR_WORKSPACE;
+  moe_status_t st = check_device();
+  if (st) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  MOE_CU(cudaMemsetAsync(send_counts, 0, (size_t)R * 4, cs));
+  if (T == 0) return MOE_OK;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* dest = reinterpret_cast<int32_t*>(w + o_dest);
+  MOE_CU(moe::launch_ep_dest(topk_ids, (int)N, E, E / R, dest, send_counts, dev_status, cs));
+  // slots in destination-rank order: align & sort with the ranks as experts and blocks of one slot
+  st = run_align(dest, T, k, R, 1, order, reinterpret_cast<int32_t*>(w + o_eids),
+                 reinterpret_cast<int32_t*>(w + o_np), w + o_al, dev_status, cs);
+  if (st) return st;
+  MOE_CU(moe::launch_ep_local_ids(topk_ids, order, (int)N, E / R, local_ids, cs));
+  return MOE_OK;
+}
+
+moe_status_t moe_permute_rows(const void* src, int row_bytes, const int32_t* map, int n, int div, int src_rows,
+                              void* dst, void* stream) {
+  if (n < 0 || div < 1 || src_rows < 0 || row_bytes <= 0 || row_bytes % 16) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!src || !map || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_permute_rows(src, row_bytes, map, n, div, src_rows, false, dst, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status_t moe_scatter_rows(const void* src, int row_bytes, const int32_t* map, int n, int dst_rows, void* dst,
+                              void* stream) {
+  if (n < 0 || dst_rows < 0 || row_bytes <= 0 || row_bytes % 16) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!src || !map || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st) return st;
+  MOE_CU(moe::launch_permute_rows(src, row_bytes, map, n, 1, dst_rows, true, dst, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
 moe_status_t moe_mx_tile_scales(const uint8_t* sf, long long rows, int K, uint8_t* out, void* stream) {
   if (rows < 0 || K < 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
   if (rows == 0 || K == 0) return MOE_OK;

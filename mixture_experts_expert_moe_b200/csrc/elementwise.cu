@@ -493,3 +493,83 @@ cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, 
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Expert-parallel helpers: destination rank of every slot (and the number of
+// slots per rank), the local expert ids of the slots in rank order, and row
+// permutations by an index map.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) ep_dest_kernel(const int32_t* __restrict__ ids, int N, int E, int E_loc,
+                                                      int32_t* __restrict__ dest, int32_t* __restrict__ counts,
+                                                      int32_t* status) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+    const int e = ids[i];
+    if (e < 0 || e >= E) {
+      dev_flag(status, MOE_DEV_BAD_EXPERT_ID);
+      dest[i] = -1;                 // align & sort skips it and flags it again
+      continue;
+    }
+    const int r = e / E_loc;
+    dest[i] = r;
+    atomicAdd(counts + r, 1);
+  }
+}
+
+__global__ void __launch_bounds__(256) ep_local_ids_kernel(const int32_t* __restrict__ ids,
+                                                           const int32_t* __restrict__ order, int N, int E_loc,
+                                                           int32_t* __restrict__ local_ids) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+    const int s = order[i];
+    local_ids[i] = s >= 0 && s < N ? ids[s] % E_loc : 0;
+  }
+}
+
+// dst row i = src row map[i] / div (gather) or dst row map[i] = src row i (scatter); 16-byte vectors, warp per row
+template <bool kScatter>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restrict__ src, int vec,
+                                                           const int32_t* __restrict__ map, int n, int div,
+                                                           int limit, uint4* __restrict__ dst) {
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+    const int m = map[i] / div;
+    if (m < 0 || m >= limit) continue;          // out-of-range map entries move nothing
+    const uint4* s = src + (long long)(kScatter ? i : m) * vec;
+    uint4* d = dst + (long long)(kScatter ? m : i) * vec;
+    for (int c = lane; c < vec; c += 32) d[c] = __ldg(s + c);
+  }
+}
+
+static int grid_for(long long n, int per_block) {
+  const long long need = (n + per_block - 1) / per_block;
+  const long long cap = (long long)sm_count() * 16;
+  return (int)(need < 1 ? 1 : (need < cap ? need : cap));
+}
+
+cudaError_t launch_ep_dest(const int32_t* ids, int N, int E, int E_loc, int32_t* dest, int32_t* counts,
+                           int32_t* status, cudaStream_t s) {
+  if (N == 0) return cudaSuccess;
+  ep_dest_kernel<<<grid_for(N, 256), 256, 0, s>>>(ids, N, E, E_loc, dest, counts, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_local_ids(const int32_t* ids, const int32_t* order, int N, int E_loc, int32_t* local_ids,
+                                cudaStream_t s) {
+  if (N == 0) return cudaSuccess;
+  ep_local_ids_kernel<<<grid_for(N, 256), 256, 0, s>>>(ids, order, N, E_loc, local_ids);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows(const void* src, int row_bytes, const int32_t* map, int n, int div, int limit,
+                                bool scatter, void* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int g = grid_for(n, 8);
+  if (scatter)
+    permute_rows_kernel<true><<<g, 256, 0, s>>>((const uint4*)src, row_bytes / 16, map, n, div, limit, (uint4*)dst);
+  else
+    permute_rows_kernel<false><<<g, 256, 0, s>>>((const uint4*)src, row_bytes / 16, map, n, div, limit, (uint4*)dst);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -70,6 +70,16 @@ cudaError_t launch_mx_quant_rows(const void* src, const int32_t* sorted, int N, 
 cudaError_t launch_mx_tile_scales(const uint8_t* in, long long rows, int K, uint8_t* out, cudaStream_t s);
 cudaError_t launch_quant_division_check(unsigned long long* counts, unsigned int* first_bad, cudaStream_t s);
 cudaError_t launch_cast_bf16(const float* src, long long n, void* dst, cudaStream_t s);
+// expert parallelism: dest[i] = ids[i] / E_loc, counts[dest] += 1 (counts zeroed by the caller)
+cudaError_t launch_ep_dest(const int32_t* ids, int N, int E, int E_loc, int32_t* dest, int32_t* counts,
+                           int32_t* status, cudaStream_t s);
+// local_ids[i] = ids[order[i]] % E_loc
+cudaError_t launch_ep_local_ids(const int32_t* ids, const int32_t* order, int N, int E_loc, int32_t* local_ids,
+                                cudaStream_t s);
+// gather: dst row i = src row map[i] / div; scatter: dst row map[i] / div = src row i (rows of row_bytes,
+// a multiple of 16; map entries whose row falls outside [0, limit) move nothing)
+cudaError_t launch_permute_rows(const void* src, int row_bytes, const int32_t* map, int n, int div, int limit,
+                                bool scatter, void* dst, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const float* w, int T, int k, int H, void* out, bool bf16,
                            cudaStream_t s);
 
