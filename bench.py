@@ -395,6 +395,47 @@ def backward_report(m, cfg, steps, warmup, dev, pk):
             "note": "dW13/dW2 in fp32 for all experts; gate/up recomputed; eager launches"}
 
 
+def ep_report(m, cfg, steps, warmup, dev):
+    """The expert-parallel layer (ep.py) over a one-rank NCCL group on this GPU:
+    gating, routing to ranks, permute, the exchange (trivial with one rank),
+    the grouped FFN over the received rows, the reverse exchange, un-permute
+    and combine, next to moe_forward on the same inputs (eager launches both).
+    With one rank the exchange moves nothing across GPUs: this measures the
+    per-rank steps' overhead, not the cost of the all-to-alls."""
+    import socket
+    import torch.distributed as dist
+    from mixture_experts_expert_moe_b200.ep import EPMoELayer
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1, device_id=dev)
+    try:
+        d, layer = build_layer(m, cfg, dev)
+        ep = EPMoELayer(d["w13"], d["w2"], cfg.E, cfg.k, cfg.bm)
+
+        def timed(fn):
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(steps):
+                fn()
+            t1.record()
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / steps
+
+        ms_ep = timed(lambda: ep(d["x"], d["logits"]))
+        ms_fw = timed(lambda: layer(d["x"], d["logits"]))
+        del d, layer, ep
+        torch.cuda.empty_cache()
+        return {"workload": "expert-parallel layer, 1 rank: " + workload_name(cfg, "bf16"), "ms_per_step": ms_ep,
+                "tokens_per_s": cfg.T / (ms_ep * 1e-3), "moe_forward_ms_per_step": ms_fw,
+                "note": "one NCCL rank: the all-to-alls move nothing; eager launches; split sizes read on the host"}
+    finally:
+        dist.destroy_process_group()
+
+
 def bm_sweep(m, cfg, steps, warmup, dev, pk, sizes=(32, 64, 128)):
     """The layer at several block sizes (routing and values unchanged; the
     padding and the GEMM token groups change), in bf16 and a8w8, each
@@ -549,6 +590,10 @@ def run_ours(args):
         extra["deepseek_mx"] = [layer_report(m, cfg.with_(mx=fmt), 30, 3, dev, pk, fmt)[0]
                                 for fmt in ("mxfp4", "mxfp8")]
         extra["backward"] = backward_report(m, cfg, 10, 3, dev, pk)
+        try:
+            extra["expert_parallel"] = ep_report(m, cfg, 20, 3, dev)
+        except Exception as exc:      # a process-group set-up problem must not cost the bench line
+            extra["expert_parallel"] = {"error": str(exc)[:300]}
         extra["align_sort"] = align_report(m, dev, pk, ALIGN_CONFIG["T"])
         extra["align_sort_large"] = align_report(m, dev, pk, 1 << 22, iters=20)
     cpu = None
@@ -758,6 +803,9 @@ def run_only(args):
             elif q.startswith("E"):
                 cfg = cfg.with_(E=int(q[1:]))
         print(json.dumps(backward_report(m, cfg, steps, warmup, dev, pk)))
+        return
+    if parts[0] == "ep":          # ep_<config>: the expert-parallel layer over one rank
+        print(json.dumps(ep_report(m, CONFIGS[parts[1]], steps, warmup, dev)))
         return
     if parts[0] == "align":
         print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
