@@ -255,8 +255,10 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   // ---- (P) stable placement ------------------------------------------------
   // Ranks: the lowest lane of each group of equal ids takes the group's
   // positions with one shared-memory atomicAdd on the warp's row (it returns
-  // the running count) and shares it by a shuffle.  The warp's atomics reach
-  // its row in issue order, so equal ids keep the order of the sub-steps.
+  // the running count) and shares it by a shuffle.  Leaders of one expert in
+  // consecutive sub-steps can be different lanes: a __syncwarp between the
+  // sub-steps orders their atomics (it is a memory fence among the warp's
+  // lanes), so equal ids keep the order of the sub-steps.
   {
     int key[kSub], nxt[kSub];
     if (w_begin < w_end) load_raw(p.ids, w_begin, w_end, lane, key);
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
         if (kq >= 0 && lane == leader) old = atomicAdd(&my[kq], __popc(peers));
         old = __shfl_sync(0xffffffffu, old, leader);
         dest[q] = kq >= 0 ? s_base[kq] + old + __popc(peers & lanemask_lt()) : -1;
+        __syncwarp();
       }
 #pragma unroll
       for (int q = 0; q < kSub; ++q)
