@@ -70,7 +70,15 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1, MOE_F32 = 2, MOE_MXFP8 = 3, MOE_M
 /* Device-side status bits (OR-ed into *dev_status). */
 #define MOE_DEV_BAD_EXPERT_ID 0x1  /* an expert id outside [0, E): slot skipped */
 #define MOE_DEV_TIMEOUT       0x2  /* a bounded wait ran out; outputs unspecified */
-#define MOE_DEV_BAD_PLAN      0x4  /* routing metadata inconsistent with sizes  */
+#define MOE_DEV_BAD_PLAN      0x4  /* routing metadata inconsistent with sizes,
+                                      or an expert's blocks not one run in
+                                      expert_ids: no GEMM tile runs          */
+#define MOE_DEV_BOUNDS        0x10 /* libraries built with MOE_DEBUG only
+                                      (libmoe_b200_debug.so): an index a kernel
+                                      computed or read fell outside its buffer
+                                      (a negative sorted id, a GEMM tile past
+                                      num_post); the access was skipped, and a
+                                      GEMM CTA stopped at its tile */
 #define MOE_DEV_DRAIN_TIMEOUT 0x8  /* after a timeout, a GEMM CTA also gave up
                                       waiting for its own copies or MMAs in
                                       flight before freeing its tensor memory:
@@ -183,8 +191,10 @@ MOE_API moe_status_t moe_align_sort_noalloc(const int32_t* topk_ids, int T, int 
  * activations with bf16 in/out); GC-MoE abstract (fused SwiGLU and
  * requantisation between the two GEMMs).
  *
- * For every sorted row r < num_post with slot s = sorted_ids[r] != T*k and
- * expert e = expert_ids[r / block_size], token t = s / k:
+ * For every sorted row r < num_post with slot s = sorted_ids[r] in [0, T*k)
+ * and expert e = expert_ids[r / block_size], token t = s / k (other ids are
+ * padding: T*k as moe_align_sort writes it; a negative id is an error that
+ * the debug build reports as MOE_DEV_BOUNDS, and both builds skip the row):
  *   BF16:  g = Wg[e] x_t, u = Wu[e] x_t (fp32 accumulation),
  *          h = bf16(silu(g) * u), y_s = Wd[e] h
  *   FP8:   (q_x, s_x) = e4m3 per-token quantisation of x_t (s = amax/448),

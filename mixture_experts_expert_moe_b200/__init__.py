@@ -14,11 +14,14 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+# MOE_B200_LIB selects another build of the same ABI (libmoe_b200_debug.so:
+# kernels with index checks that report MOE_DEV_BOUNDS)
+LIB_PATH = os.environ.get("MOE_B200_LIB") or os.path.join(_PKG, "libmoe_b200.so")
 
 MOE_BF16, MOE_FP8_E4M3, MOE_F32, MOE_MXFP8, MOE_MXFP4 = 0, 1, 2, 3, 4
 _MX_TYPES = {"mxfp8": MOE_MXFP8, "mxfp4": MOE_MXFP4}
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_PLAN, MOE_DEV_DRAIN_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+MOE_DEV_BOUNDS = 0x10   # debug builds only: an out-of-range index was skipped
 STAGES = ["gate", "align", "plan", "gather", "gateup", "requant", "down", "combine"]
 
 EXPORTED = [

@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
       }
 #pragma unroll
       for (int q = 0; q < kSub; ++q)
-        if (dest[q] >= 0) p.sorted[dest[q]] = (int)(base + q * 32 + lane);
+        if (dest[q] >= 0 && MOE_IN_BOUNDS(dest[q] < p.N + p.E * (p.bm - 1), p.status))
+          p.sorted[dest[q]] = (int)(base + q * 32 + lane);
 #pragma unroll
       for (int q = 0; q < kSub; ++q) key[q] = nxt[q];
     }

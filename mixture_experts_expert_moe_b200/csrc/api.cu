@@ -5,6 +5,8 @@
 #include <cstring>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 
 namespace {
@@ -31,6 +33,15 @@ inline moe_status_t cuda_fail(cudaError_t e, const char* where) { return moe::re
   } while (0)
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// An NVTX range over a scope (entry points and the forward's stages show up
+// by name in Nsight Systems / Compute timelines; a no-op without a tool).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 struct Carver {
   size_t off = 0;
@@ -231,10 +242,13 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   const int P = (int)s.P, N = (int)s.N;
   const int R = (int)s.rows_max;   // grid size of the row kernels (they read num_post on the device)
 
-  if (!plan_ready)
+  if (!plan_ready) {
+    NvtxRange nr("moe: tile plan");
     MOE_CU(moe::launch_plan(expert_ids, num_post, sorted, N, P, s.E, s.bm, s.tn, s.I / 128, (s.H + 255) / 256, plan,
                             status, stream));
+  }
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
+  nvtxRangePushA("moe: gather");
   if (s.mx) {
     // every sorted row MX-quantises its token (codes + a scale per 32 elements)
     MOE_CU(moe::launch_mx_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, reinterpret_cast<uint8_t*>(sA),
@@ -249,6 +263,7 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   } else {
     MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, R, N, s.k, s.H * 2, A, nullptr, stream));
   }
+  nvtxRangePop();
   MOE_CU(record(ev, MOE_STAGE_GATHER + 1, stream));
 
   moe::GemmLaunch g1 = {};
@@ -277,7 +292,11 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   g1.p.status = status;
   g1.p.timeout_ns = moe::kDefaultTimeoutNs;
   g1.p.tile_counter = plan + moe::plan_counter(s.E, true);
-  int r = moe::launch_grouped_gemm(g1, stream);
+  int r;
+  {
+    NvtxRange nr("moe: gate/up GEMM");
+    r = moe::launch_grouped_gemm(g1, stream);
+  }
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
 
@@ -311,7 +330,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   g2.p.tile_counter = plan + moe::plan_counter(s.E, false);
   g2.p.comb_out = comb_out;   // non-null: out32[t] += w * y in the epilogue, y is not written
   g2.p.comb_w = comb_w;
-  r = moe::launch_grouped_gemm(g2, stream);
+  {
+    NvtxRange nr("moe: down GEMM");
+    r = moe::launch_grouped_gemm(g2, stream);
+  }
   if (r) return gemm_fail(r, "down GEMM");
   MOE_CU(record(ev, MOE_STAGE_DOWN + 1, stream));
   return MOE_OK;
@@ -411,6 +433,7 @@ int moe_version(void) { return MOE_ABI_VERSION; }
 
 moe_status_t moe_topk_gate(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
                            int n_shared, int32_t* topk_ids, float* topk_w, void* stream) {
+  NvtxRange nvtx_("moe_topk_gate");
   if (T < 0 || E < 1 || k < 1 || k > E || n_shared < 0 || k + n_shared > 32 || E + n_shared > 1024)
     return MOE_ERR_INVALID_ARG;
   if (bias_mode != MOE_BIAS_LOGITS && bias_mode != MOE_BIAS_SELECT) return MOE_ERR_INVALID_ARG;
@@ -435,6 +458,7 @@ moe_status_t moe_align_sort_sizes(int T, int k, int E, int block_size, size_t* P
 moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int k, int E, int block_size, int32_t* sorted_ids,
                             int32_t* expert_ids, int32_t* num_post, void* ws, size_t ws_bytes,
                             int32_t* dev_status, void* stream) {
+  NvtxRange nvtx_("moe_align_sort");
   if (!align_args_ok(T, k, E, block_size)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids || !expert_ids || !num_post || !ws || (T > 0 && !topk_ids)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < align_ws_bytes(E)) return MOE_ERR_WORKSPACE;
@@ -455,6 +479,7 @@ moe_status_t moe_ffn_workspace(const moe_ffn_args* a, size_t* ws_bytes) {
 
 moe_status_t moe_grouped_ffn(const moe_ffn_args* a, float* y, void* ws, size_t ws_bytes, int32_t* dev_status,
                              void* stream) {
+  NvtxRange nvtx_("moe_grouped_ffn");
   if (!a) return MOE_ERR_INVALID_ARG;
   FfnShape s;
   moe_status_t st = ffn_shape(a->T, a->H, a->I, a->E, a->k, a->block_size, a->wdtype, a->tile_tokens, &s);
@@ -475,6 +500,7 @@ moe_status_t moe_grouped_ffn(const moe_ffn_args* a, float* y, void* ws, size_t w
 
 moe_status_t moe_combine(const float* y, const float* topk_w, int T, int k, int H, void* out, int out_dtype,
                          void* stream) {
+  NvtxRange nvtx_("moe_combine");
   if (T < 0 || k < 1 || H < 1 || H % 4) return MOE_ERR_INVALID_ARG;
   if (out_dtype != MOE_BF16 && out_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -541,6 +567,7 @@ moe_status_t moe_forward_workspace(const moe_forward_args* a, size_t* ws_bytes) 
 
 moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
                          void* stream) {
+  NvtxRange nvtx_("moe_forward");
   if (!a) return MOE_ERR_INVALID_ARG;
   FfnShape s;
   moe_status_t st = forward_shape(a, &s);
@@ -571,8 +598,11 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   // gate, align&sort and the GEMM tile plan are one launch: stages 0..2 end together
   uint8_t* ffn_ws = w + L.ffn;
   int32_t* plan = reinterpret_cast<int32_t*>(ffn_ws + ffn_ws_layout(s).plan);
-  st = run_route(s, a->n_shared, a->bias_mode == MOE_BIAS_SELECT, a->logits, a->bias, ids, tw, sorted, eids, npost,
-                 w + L.align, plan, dev_status, cs);
+  {
+    NvtxRange nr("moe: route (gate, align & sort, plan)");
+    st = run_route(s, a->n_shared, a->bias_mode == MOE_BIAS_SELECT, a->logits, a->bias, ids, tw, sorted, eids,
+                   npost, w + L.align, plan, dev_status, cs);
+  }
   if (st) return st;
   MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));
   MOE_CU(record(ev, MOE_STAGE_ALIGN + 1, cs));
@@ -581,6 +611,7 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   const FfnWeights W = {a->w13, a->w13_scale, a->w2, a->w2_scale, a->w13_mx_scale, a->w2_mx_scale};
   st = run_ffn(s, a->x, W, sorted, eids, npost, y, ffn_ws, dev_status, cs, ev, /*plan_ready=*/true, out32, tw);
   if (st) return st;
+  NvtxRange nr_combine("moe: combine");
   if (fused) {
     if (out_bf16) MOE_CU(moe::launch_cast_bf16(out32, (long long)s.T * s.H, a->out, cs));
   } else {
@@ -657,6 +688,7 @@ moe_status_t moe_backward_workspace(const moe_backward_args* a, size_t* ws_bytes
 
 moe_status_t moe_backward(const moe_backward_args* a, void* ws, size_t ws_bytes, int32_t* dev_status,
                           void* stream) {
+  NvtxRange nvtx_("moe_backward");
   if (!a) return MOE_ERR_INVALID_ARG;
   FfnShape s;
   moe_status_t st = bwd_shape(a, &s);
@@ -778,6 +810,7 @@ moe_status_t moe_ep_route_workspace(int T, int k, int R, size_t* ws_bytes) {
 
 moe_status_t moe_ep_route(const int32_t* topk_ids, int T, int k, int E, int R, int32_t* order, int32_t* send_counts,
                           int32_t* local_ids, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  NvtxRange nvtx_("moe_ep_route");
   if (!align_args_ok(T, k, R, 1) || E < R || E % R) return MOE_ERR_INVALID_ARG;
   if (!send_counts || (T > 0 && (!topk_ids || !order || !local_ids || !ws))) return MOE_ERR_INVALID_ARG;
   const long long N = (long long)T * k;

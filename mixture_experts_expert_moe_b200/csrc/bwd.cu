@@ -143,6 +143,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
         const BwdTile bt = bwd_tile(p, t, s_pref, s_perm, s_start, s_rows, s_groups, s_prow);
         if (bt.skip) continue;
+        if (!MOE_IN_BOUNDS(bt.e >= 0 && bt.e < E && bt.r0 >= 0 && bt.r0 + bt.nrows <= p.plan[PLAN_NUM_POST],
+                           p.status)) {
+          *abort_flag = 2;     // every role stops at its next wait (2: not a timeout)
+          ok = false;
+          break;
+        }
         // A rows / columns of the two sub-tiles
         int a0, a1;            // K-major: weight rows; MN-major: first feature column
         bool has1 = paired;
@@ -318,14 +324,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           float g[16], u[16];
           const bool in = lane < 16 && c + lane < bt.nrows;
           const int slot_l = in ? __ldg(p.sorted + bt.r0 + c + lane) : p.n_slots;
-          const float w_l = slot_l < p.n_slots ? __ldg(p.topk_w + slot_l) : 0.f;
+          const float w_l = (unsigned)slot_l < (unsigned)p.n_slots ? __ldg(p.topk_w + slot_l) : 0.f;
           tmem_ld16(tb + c, g);
           tmem_ld16(tb + p.tn + c, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int slot = __shfl_sync(0xffffffffu, slot_l, i);
             const float w = __shfl_sync(0xffffffffu, w_l, i);
-            if (c + i < bt.nrows && slot < p.n_slots) {      // uniform across the warp
+            // uniform across the warp
+            if (c + i < bt.nrows && MOE_IN_BOUNDS(slot >= 0, p.status) && (unsigned)slot < (unsigned)p.n_slots) {
               const size_t row = (size_t)(bt.r0 + c + i);
               const float gv = g[i], uv = u[i];
               const float s = 1.f / (1.f + expf(-gv));
@@ -360,7 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int slot = __shfl_sync(0xffffffffu, slot_l, i);
-            if (c + i < bt.nrows && slot < p.n_slots) {
+            if (c + i < bt.nrows && MOE_IN_BOUNDS(slot >= 0, p.status) && (unsigned)slot < (unsigned)p.n_slots) {
               float* row = p.dx + (size_t)(slot / p.k) * p.n_out;
               red_add_f32(row + n0, v0[i], pol);
               if (has1) red_add_f32(row + n1, v1[i], pol);
@@ -389,7 +396,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) dev_flag(p.status, MOE_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && *abort_flag == 1) dev_flag(p.status, MOE_DEV_TIMEOUT);
   if (threadIdx.x == 0 && *s_drain_fail) dev_flag(p.status, MOE_DEV_DRAIN_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();

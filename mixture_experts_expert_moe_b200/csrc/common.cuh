@@ -24,6 +24,19 @@ __device__ __forceinline__ void dev_flag(int32_t* st, int bits) {
   if (st) atomicOr(st, bits);
 }
 
+// Bounds checks of the MOE_DEBUG build (the stand-in for a memory checker):
+// MOE_IN_BOUNDS(cond, status) is cond, and flags MOE_DEV_BOUNDS when cond is
+// false; without MOE_DEBUG it is true and compiles away.
+#ifdef MOE_DEBUG
+__device__ __forceinline__ bool moe_in_bounds(bool ok, int32_t* st) {
+  if (!ok) dev_flag(st, MOE_DEV_BOUNDS);
+  return ok;
+}
+#define MOE_IN_BOUNDS(cond, st) moe_in_bounds((cond), (st))
+#else
+#define MOE_IN_BOUNDS(cond, st) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

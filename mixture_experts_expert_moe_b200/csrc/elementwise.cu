@@ -53,15 +53,15 @@ cudaError_t launch_topk_gate(const float* logits, const float* bias, bool select
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
                                                           const float* __restrict__ src_scale,
                                                           const int32_t* __restrict__ sorted,
-                                                          const int32_t* __restrict__ num_post, int N, int k,
-                                                          int vec, uint4* __restrict__ dst,
+                                                          const int32_t* __restrict__ num_post, int P, int N,
+                                                          int k, int vec, uint4* __restrict__ dst,
                                                           float* __restrict__ dst_scale) {
-  const int np = *num_post;
+  const int np = min(*num_post, P);   // an invalid num_post (flagged by the plan) stays inside the buffers
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < np; r += gridDim.x * wpb) {
     const int slot = __ldg(sorted + r);
-    const long long t = slot < N ? slot / k : -1;
+    const long long t = (unsigned)slot < (unsigned)N ? slot / k : -1;   // padding, or an invalid id: zeros
     const uint4* row = t >= 0 ? src + t * vec : nullptr;
     uint4* out = dst + (long long)r * vec;
     int c = lane;
@@ -172,7 +172,7 @@ __device__ __forceinline__ void quant_store(const uint4 (&v)[V], const RowScale&
 __device__ __forceinline__ long long quant_src_row(const int32_t* sorted, int r, int N, int k) {
   if (!sorted) return r;
   const int slot = __ldg(sorted + r);
-  return slot < N ? slot / k : -1;
+  return (unsigned)slot < (unsigned)N ? slot / k : -1;
 }
 
 template <int VPL>
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
                                                               const int32_t* __restrict__ nrows_dev, int nrows,
                                                               int vec, uint2* __restrict__ q,
                                                               float* __restrict__ scale) {
-  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int n = nrows_dev ? min(*nrows_dev, nrows) : nrows;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t row_bytes = (uint32_t)vec * 16u;
   uint8_t* buf = smq + (size_t)warp * nb * row_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smq + (size_t)W * nb * row_bytes) + warp * nb;
-  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int n = nrows_dev ? min(*nrows_dev, nrows) : nrows;
   const int first = blockIdx.x * W + warp, stride = gridDim.x * W;
   if (lane == 0) {
     for (int b = 0; b < nb; ++b) mbar_init(&bars[b], 1);
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(256, 1)
   auto source = [&](int r) -> long long {
     if (!kGather) return r;
     const int slot = __ldg(sorted + r);
-    return slot < N ? slot / k : -1;
+    return (unsigned)slot < (unsigned)N ? slot / k : -1;
   };
   // lane 0: the i-th row of this warp into buffer i % nb (a padding row only completes the phase)
   auto issue = [&](int i) {
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __re
                                                                const int32_t* __restrict__ nrows_dev, int nrows,
                                                                int vec, uint2* __restrict__ q,
                                                                float* __restrict__ scale) {
-  const int n = nrows_dev ? *nrows_dev : nrows;
+  const int n = nrows_dev ? min(*nrows_dev, nrows) : nrows;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
@@ -346,8 +346,8 @@ static int warp_rows_grid(long long rows) {
 cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,
                                const int32_t* num_post, int P, int N, int k, int row_bytes, void* dst,
                                float* dst_scale, cudaStream_t s) {
-  gather_rows_kernel<<<warp_rows_grid(P), 256, 0, s>>>((const uint4*)src, src_scale, sorted, num_post, N, k,
-                                                        row_bytes / 16, (uint4*)dst, dst_scale);
+  gather_rows_kernel<<<warp_rows_grid(P), 256, 0, s>>>((const uint4*)src, src_scale, sorted, num_post, P, N,
+                                                        k, row_bytes / 16, (uint4*)dst, dst_scale);
   return cudaGetLastError();
 }
 
@@ -533,8 +533,9 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
                                                            int limit, uint4* __restrict__ dst) {
   const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
   for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
-    const int m = map[i] / div;
-    if (m < 0 || m >= limit) continue;          // out-of-range map entries move nothing
+    const int v = map[i];
+    const int m = v / div;
+    if (v < 0 || m >= limit) continue;          // out-of-range map entries move nothing
     const uint4* s = src + (long long)(kScatter ? i : m) * vec;
     uint4* d = dst + (long long)(kScatter ? m : i) * vec;
     for (int c = lane; c < vec; c += 32) d[c] = __ldg(s + c);

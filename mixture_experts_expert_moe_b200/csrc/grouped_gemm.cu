@@ -47,14 +47,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int bm, int tn, int nw_gu, int nw_dn,
                                                     int32_t* __restrict__ plan, int32_t* status) {
   extern __shared__ int sm[];
-  int* s_first = sm;        // [E] first block of expert
+  int* s_first = sm;        // [E] first block of expert (-1: none)
   int* s_nblk = sm + E;     // [E] blocks of expert -> token groups
   int* sc = sm + 2 * E;     // [3E + 2] scratch of finish_plan
+  int* s_bad = sm + 5 * E + 2;
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) {
-    s_first[e] = 0;
+    s_first[e] = -1;
     s_nblk[e] = 0;
   }
+  if (tid == 0) *s_bad = 0;
   __syncthreads();
   int np = *num_post;
   if (np < 0 || np > P || np % bm != 0) {
@@ -69,16 +71,22 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
       continue;
     }
     atomicAdd(&s_nblk[e], 1);
-    if (b == 0 || expert_ids[b - 1] != e) s_first[e] = b;
+    // the blocks of an expert form one run (a second run start would give a
+    // segment reaching past num_post): anything else is an invalid plan
+    if ((b == 0 || expert_ids[b - 1] != e) && atomicExch(&s_first[e], b) != -1) {
+      dev_flag(status, MOE_DEV_BAD_PLAN);
+      *s_bad = 1;
+    }
   }
   __syncthreads();
+  if (*s_bad) np = 0;       // an invalid plan runs no tiles
   for (int e = tid; e < E; e += blockDim.x) {
-    const int rows = s_nblk[e] * bm;
-    const int start = s_first[e] * bm;
+    const int rows = np ? s_nblk[e] * bm : 0;
+    const int start = rows ? s_first[e] * bm : 0;
     // padding (slot id >= N) fills the end of the segment: count it in the last block
     int real = rows;
     for (int i = rows - 1; i >= 0 && i >= rows - bm; --i) {
-      if (sorted[start + i] < N) break;
+      if ((unsigned)sorted[start + i] < (unsigned)N) break;
       --real;
     }
     plan[plan_start(E) + e] = start;
@@ -92,7 +100,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 
 cudaError_t launch_plan(const int32_t* expert_ids, const int32_t* num_post, const int32_t* sorted, int N, int P,
                         int E, int bm, int tn, int nw_gu, int nw_dn, int32_t* plan, int32_t* status, cudaStream_t s) {
-  plan_kernel<<<1, 1024, (5 * E + 2) * sizeof(int), s>>>(expert_ids, num_post, sorted, N, P, E, bm, tn, nw_gu,
+  plan_kernel<<<1, 1024, (5 * E + 3) * sizeof(int), s>>>(expert_ids, num_post, sorted, N, P, E, bm, tn, nw_gu,
                                                          nw_dn, plan, status);
   return cudaGetLastError();
 }
@@ -222,6 +230,12 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
         mbar_arrive(&t_full[slot]);
         if (t >= n_tiles) break;
         const TileInfo ti = decode_tile(t, s_pref, s_perm, s_start, s_rows, s_groups, E, p.tn);
+        if (!MOE_IN_BOUNDS(ti.e >= 0 && ti.e < E && ti.r0 >= 0 && ti.r0 + ti.nrows <= p.plan[PLAN_NUM_POST],
+                           p.status)) {
+          *abort_flag = 2;     // every role stops at its next wait (2: not a timeout)
+          ok = false;
+          break;
+        }
         int row0, row1;
         bool has1 = true;
         if (p.gateup) {
@@ -443,7 +457,9 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
           const bool in = lane < 16 && c + lane < ti.nrows;
           const int slot_l = in ? __ldg(p.sorted + ti.r0 + c + lane) : p.n_slots;
           const float sa_l = (p.fp8 && in) ? __ldg(p.a_scale + ti.r0 + c + lane) : 1.f;
-          const float wt_l = (fused && slot_l < p.n_slots) ? __ldg(p.comb_w + slot_l) : 0.f;
+          // a negative slot id is invalid (debug builds report it); like padding it writes nothing
+          const bool valid_l = (unsigned)slot_l < (unsigned)p.n_slots;
+          const float wt_l = (fused && valid_l) ? __ldg(p.comb_w + slot_l) : 0.f;
           tmem_ld16(tb + c, v0);
           if (has1) tmem_ld16(tb + p.tn + c, v1);
 #pragma unroll
@@ -451,7 +467,7 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
             const int slot = __shfl_sync(0xffffffffu, slot_l, i);
             const float sa = __shfl_sync(0xffffffffu, sa_l, i);
             const float wt = __shfl_sync(0xffffffffu, wt_l, i);
-            if (c + i < ti.nrows && slot < p.n_slots) {
+            if (c + i < ti.nrows && MOE_IN_BOUNDS(slot >= 0, p.status) && (unsigned)slot < (unsigned)p.n_slots) {
               const float a0 = p.fp8 ? v0[i] * sa * sw0 : v0[i];
               const float a1 = p.fp8 ? v1[i] * sa * sw1 : v1[i];
               if (fused) {
@@ -515,7 +531,7 @@ __global__ void __launch_bounds__(kMX ? kGemmThreadsMx : kGemmThreads, 1)
   }
 
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) dev_flag(p.status, MOE_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && *abort_flag == 1) dev_flag(p.status, MOE_DEV_TIMEOUT);
   if (threadIdx.x == 0 && *s_drain_fail) dev_flag(p.status, MOE_DEV_DRAIN_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();

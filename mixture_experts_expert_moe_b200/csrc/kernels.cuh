@@ -48,17 +48,16 @@ cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout
 // ids/w rows of k + n_shared entries (the shared experts E.. with weight 1)
 cudaError_t launch_topk_gate(const float* logits, const float* bias, bool select_only, int T, int E, int k,
                              int n_shared, int32_t* ids, float* w, cudaStream_t s);
-// dst row r = src row sorted[r]/k (row_bytes each, a multiple of 16), zero for
-// padding; with scales also dst_scale[r] = src_scale[token] (1 for padding)
+// dst row r < min(*num_post, P) = src row sorted[r]/k (row_bytes each, a
+// multiple of 16), zero for padding (an id outside [0, N)); with scales also
+// dst_scale[r] = src_scale[token] (1 for padding)
 cudaError_t launch_gather_rows(const void* src, const float* src_scale, const int32_t* sorted,
                                const int32_t* num_post, int P, int N, int k, int row_bytes, void* dst,
                                float* dst_scale, cudaStream_t s);
-// per-row E4M3 quantisation of bf16 rows of length C; rows = *nrows_dev if
-// non-null, else nrows.  With `sorted`, output row r quantises source row
-// sorted[r] / k (zero codes, scale 1 for padding slots >= N).
-// rows [0, *nrows_dev) (or [0, nrows) when nrows_dev is null; nrows bounds
-// *nrows_dev) of src [.., C] bf16 -> E4M3 codes + fp32 scales; with sorted,
-// row r quantises token sorted[r] / k (zero codes, scale 1 for padding)
+// per-row E4M3 quantisation of bf16 rows of length C: rows
+// [0, min(*nrows_dev, nrows)) (or [0, nrows) when nrows_dev is null) of
+// src [.., C] -> E4M3 codes + fp32 scales.  With `sorted`, row r quantises
+// token sorted[r] / k (zero codes, scale 1 for padding: an id outside [0, N))
 cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
                               int nrows, int C, void* q, float* scale, int32_t* status, cudaStream_t s);
 // MXFP8 quantisation of bf16 rows of length C (C % 32 == 0): E4M3 codes

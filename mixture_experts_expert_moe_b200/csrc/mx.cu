@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const uint4* __restr
     long long t = r;
     if (sorted) {
       const int slot = __ldg(sorted + r);
-      t = slot < N ? slot / k : -1;
+      t = (unsigned)slot < (unsigned)N ? slot / k : -1;
     }
     const uint4* row = t >= 0 ? src + t * vec : nullptr;
     uint2* out = codes + (long long)r * vec;

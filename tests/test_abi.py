@@ -26,6 +26,41 @@ def test_library_exports_every_declared_symbol():
     assert sorted(m.EXPORTED) == names
 
 
+def _debug_library_path():
+    from mixture_experts_expert_moe_b200 import build_lib
+    if not os.path.exists(build_lib.DEBUG_LIB):
+        build_lib.build(debug=True)
+    return build_lib.DEBUG_LIB
+
+
+def test_debug_library_exports_the_same_abi():
+    """libmoe_b200_debug.so (kernels compiled with MOE_DEBUG index checks)
+    implements the same ABI: every declared symbol and the same version."""
+    path = _debug_library_path()
+    assert os.path.abspath(path) != os.path.abspath(m.LIB_PATH)
+    lib = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    lib.moe_version.restype = ctypes.c_int
+    assert lib.moe_version() == m.ABI_VERSION
+    assert m.MOE_DEV_BOUNDS == 0x10
+    text = open(HEADER).read()
+    assert re.search(r"#define MOE_DEV_BOUNDS\s+0x10\b", text)
+
+
+def test_library_path_override_selects_the_debug_build():
+    import subprocess
+    import sys
+    path = _debug_library_path()
+    env = dict(os.environ, MOE_B200_LIB=path)
+    code = ("import mixture_experts_expert_moe_b200 as m; lib = m.load_library(); "
+            "print(m.LIB_PATH); print(lib.moe_version())")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == [path, str(m.ABI_VERSION)]
+
+
 def test_status_strings_and_version():
     lib = m.load_library()
     assert lib.moe_status_string(0) == b"MOE_OK"
