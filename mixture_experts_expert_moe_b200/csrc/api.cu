@@ -255,10 +255,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
                                      stream));
   } else if (s.fp8 && N <= kFusedQuantSlots) {
     // few slots: each sorted row quantises its token directly (one launch)
-    MOE_CU(moe::launch_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, sA, status, stream));
+    MOE_CU(moe::launch_quant_rows(x, sorted, /*gather=*/true, N, s.k, num_post, R, s.H, A, sA, status, stream));
   } else if (s.fp8) {
     // quantise each token once, then gather codes and scales into sorted order
-    MOE_CU(moe::launch_quant_rows(x, nullptr, N, s.k, nullptr, s.T, s.H, xq, sx, status, stream));
+    MOE_CU(moe::launch_quant_rows(x, nullptr, false, N, s.k, nullptr, s.T, s.H, xq, sx, status, stream));
     MOE_CU(moe::launch_gather_rows(xq, sx, sorted, num_post, R, N, s.k, s.H, A, sA, stream));
   } else {
     MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, R, N, s.k, s.H * 2, A, nullptr, stream));
@@ -300,7 +300,10 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
   if (r) return gemm_fail(r, "gate/up GEMM");
   MOE_CU(record(ev, MOE_STAGE_GATEUP + 1, stream));
 
-  if (s.fp8) MOE_CU(moe::launch_quant_rows(h, nullptr, N, s.k, num_post, R, s.I, hq, sH, status, stream));
+  // padding rows of h are skipped: the gate/up GEMM does not write them, and
+  // the down GEMM stores no column of a padding slot
+  if (s.fp8)
+    MOE_CU(moe::launch_quant_rows(h, sorted, /*gather=*/false, N, s.k, num_post, R, s.I, hq, sH, status, stream));
   MOE_CU(record(ev, MOE_STAGE_REQUANT + 1, stream));
 
   moe::GemmLaunch g2 = {};

@@ -167,31 +167,31 @@ __device__ __forceinline__ void quant_store(const uint4 (&v)[V], const RowScale&
   }
 }
 
-// gather (optional): row r quantises token sorted[r] / k of src (padding
-// rows: zero codes, scale 1) instead of src row r.
-__device__ __forceinline__ long long quant_src_row(const int32_t* sorted, int r, int N, int k) {
+// Source row of output row r.  Without a row map: src row r.  With the
+// sorted slot ids as row map: the token sorted[r] / k (gather) or src row r,
+// and -1 for a padding row (an id outside [0, N)), which is not written:
+// nothing reads the codes of a padding row (the grouped GEMMs compute a
+// padding row's column but store none of it).
+__device__ __forceinline__ long long quant_src_row(const int32_t* sorted, bool gather, int r, int N, int k) {
   if (!sorted) return r;
   const int slot = __ldg(sorted + r);
-  return (unsigned)slot < (unsigned)N ? slot / k : -1;
+  if ((unsigned)slot < (unsigned)N) return gather ? slot / k : r;
+  return -1;
 }
 
 template <int VPL>
 __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __restrict__ src,
-                                                              const int32_t* __restrict__ sorted, int N, int k,
-                                                              const int32_t* __restrict__ nrows_dev, int nrows,
-                                                              int vec, uint2* __restrict__ q,
+                                                              const int32_t* __restrict__ sorted, bool gather,
+                                                              int N, int k, const int32_t* __restrict__ nrows_dev,
+                                                              int nrows, int vec, uint2* __restrict__ q,
                                                               float* __restrict__ scale) {
   const int n = nrows_dev ? min(*nrows_dev, nrows) : nrows;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
-    const long long sr = quant_src_row(sorted, r, N, k);
+    const long long sr = quant_src_row(sorted, gather, r, N, k);
+    if (sr < 0) continue;
     uint2* dst = q + (long long)r * vec;
-    if (sr < 0) {
-      for (int c = lane; c < vec; c += 32) dst[c] = make_uint2(0, 0);
-      if (lane == 0) scale[r] = 1.f;
-      continue;
-    }
     const uint4* row = src + sr * vec;
     uint4 v[VPL];
     float amax = 0.f;
@@ -217,9 +217,9 @@ __global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __res
 // vectors from shared memory.  Warp w of CTA c takes rows c*W + w + i*gridDim*W.
 // A wait that runs out flags MOE_DEV_TIMEOUT, lets the warp's copies in flight
 // land (bounded) and returns.
-template <bool kGather>
 __global__ void __launch_bounds__(256, 1)
-    quant_rows_bulk_kernel(const uint8_t* __restrict__ src, const int32_t* __restrict__ sorted, int N, int k,
+    quant_rows_bulk_kernel(const uint8_t* __restrict__ src, const int32_t* __restrict__ sorted, bool gather,
+                           int N, int k,
                            const int32_t* __restrict__ nrows_dev, int nrows, int vec, int nb,
                            uint2* __restrict__ q, float* __restrict__ scale, int32_t* status,
                            long long timeout_ns) {
@@ -235,12 +235,7 @@ __global__ void __launch_bounds__(256, 1)
     fence_mbar_init();
   }
   __syncwarp();
-  // source row of sorted row r: the token in gather mode (-1 for padding)
-  auto source = [&](int r) -> long long {
-    if (!kGather) return r;
-    const int slot = __ldg(sorted + r);
-    return (unsigned)slot < (unsigned)N ? slot / k : -1;
-  };
+  auto source = [&](int r) -> long long { return quant_src_row(sorted, gather, r, N, k); };
   // lane 0: the i-th row of this warp into buffer i % nb (a padding row only completes the phase)
   auto issue = [&](int i) {
     const int r = first + i * stride;
@@ -274,10 +269,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     const uint4* row = reinterpret_cast<const uint4*>(buf + (size_t)b * row_bytes);
     uint2* dst = q + (long long)r * vec;
-    if (source(r) < 0) {
-      for (int c = lane; c < vec; c += 32) dst[c] = make_uint2(0, 0);
-      if (lane == 0) scale[r] = 1.f;
-    } else {
+    if (source(r) >= 0) {   // padding rows are not written
       float amax = 0.f;
       for (int c = lane; c < vec; c += 32) amax = fmaxf(amax, absmax8(row[c]));
       amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
@@ -300,7 +292,8 @@ __global__ void __launch_bounds__(256, 1)
 
 // (the second pass re-reads the row from L1/L2).
 __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __restrict__ src,
-                                                               const int32_t* __restrict__ sorted, int N, int k,
+                                                               const int32_t* __restrict__ sorted, bool gather,
+                                                               int N, int k,
                                                                const int32_t* __restrict__ nrows_dev, int nrows,
                                                                int vec, uint2* __restrict__ q,
                                                                float* __restrict__ scale) {
@@ -308,13 +301,9 @@ __global__ void __launch_bounds__(256) quant_rows_2pass_kernel(const uint4* __re
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
-    const long long sr = quant_src_row(sorted, r, N, k);
+    const long long sr = quant_src_row(sorted, gather, r, N, k);
+    if (sr < 0) continue;
     uint2* dst = q + (long long)r * vec;
-    if (sr < 0) {
-      for (int c = lane; c < vec; c += 32) dst[c] = make_uint2(0, 0);
-      if (lane == 0) scale[r] = 1.f;
-      continue;
-    }
     const uint4* row = src + sr * vec;
     float amax = 0.f;
     for (int c = lane; c < vec; c += 32) amax = fmaxf(amax, absmax8(__ldg(row + c)));
@@ -351,8 +340,9 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
-                              int nrows, int C, void* q, float* scale, int32_t* status, cudaStream_t s) {
+cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, bool gather, int N, int k,
+                              const int32_t* nrows_dev, int nrows, int C, void* q, float* scale, int32_t* status,
+                              cudaStream_t s) {
   const int vec = C / 8;
   if (C >= 4096) {
     // long rows, staged in shared memory: W warps x nb buffers of one row
@@ -371,11 +361,11 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int
       const long long ctas = ((long long)nrows + W - 1) / W;
       const int sms = sm_count();
       const int g = (int)(ctas < sms ? ctas : sms);
-      auto kern = sorted ? quant_rows_bulk_kernel<true> : quant_rows_bulk_kernel<false>;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaError_t e = cudaFuncSetAttribute(quant_rows_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
       if (e != cudaSuccess) return e;
-      kern<<<g, 32 * W, smem, s>>>((const uint8_t*)src, sorted, N, k, nrows_dev, nrows, vec, nb, (uint2*)q, scale,
-                                   status, kDefaultTimeoutNs);
+      quant_rows_bulk_kernel<<<g, 32 * W, smem, s>>>((const uint8_t*)src, sorted, gather, N, k, nrows_dev, nrows,
+                                                     vec, nb, (uint2*)q, scale, status, kDefaultTimeoutNs);
       return cudaGetLastError();
     }
   }
@@ -383,13 +373,14 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int
   const int g = warp_rows_grid(nrows);
   const uint4* in = (const uint4*)src;
   uint2* out = (uint2*)q;
-#define MOE_QUANT(V) quant_rows_warp_kernel<V><<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale)
+#define MOE_QUANT(V) \
+  quant_rows_warp_kernel<V><<<g, 256, 0, s>>>(in, sorted, gather, N, k, nrows_dev, nrows, vec, out, scale)
   if (vpl <= 1) MOE_QUANT(1);
   else if (vpl <= 2) MOE_QUANT(2);
   else if (vpl <= 4) MOE_QUANT(4);
   else if (vpl <= 8) MOE_QUANT(8);
   else if (vpl <= 16) MOE_QUANT(16);
-  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, N, k, nrows_dev, nrows, vec, out, scale);
+  else quant_rows_2pass_kernel<<<g, 256, 0, s>>>(in, sorted, gather, N, k, nrows_dev, nrows, vec, out, scale);
 #undef MOE_QUANT
   return cudaGetLastError();
 }

@@ -13,7 +13,7 @@ struct AlignParams {
   int N;            // T*k flat slots
   int E;
   int bm;
-  int chunk;        // slots per CTA, a multiple of 32 * kAlignWarps
+  int chunk;        // slots per CTA: a multiple of 32 and of the slots per token
   int32_t* sorted;
   int32_t* expert_ids;
   int32_t* num_post;
@@ -57,11 +57,13 @@ cudaError_t launch_gather_rows(const void* src, const float* src_scale, const in
 // per-row E4M3 quantisation of bf16 rows of length C: rows
 // [0, min(*nrows_dev, nrows)) (or [0, nrows) when nrows_dev is null) of
 // src [.., C] -> E4M3 codes + fp32 scales.  With `sorted`, row r quantises
-// token sorted[r] / k (zero codes, scale 1 for padding: an id outside [0, N))
-cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
-                              int nrows, int C, void* q, float* scale, int32_t* status, cudaStream_t s);
+// token sorted[r] / k (gather) or src row r, and padding rows (an id outside
+// [0, N)) are not written.
+cudaError_t launch_quant_rows(const void* src, const int32_t* sorted, bool gather, int N, int k,
+                              const int32_t* nrows_dev, int nrows, int C, void* q, float* scale, int32_t* status,
+                              cudaStream_t s);
 // MXFP8 quantisation of bf16 rows of length C (C % 32 == 0): E4M3 codes
-// [rows, C] and E8M0 scales [rows, C/32]; rows and the row map as in
+// [rows, C] and E8M0 scales [rows, C/32]; rows and the gather row map as in
 // launch_quant_rows (padding rows: zero codes, scale code 127)
 cudaError_t launch_mx_quant_rows(const void* src, const int32_t* sorted, int N, int k, const int32_t* nrows_dev,
                                  int nrows, int C, void* codes, uint8_t* scales, cudaStream_t s);

@@ -109,6 +109,33 @@ def test_forward_parity_small(cuda_device, cfg, a8w8):
         assert_close(out.float().cpu().numpy(), ref, tol, f"{cfg.name} out {out_dtype}")
 
 
+# many experts: 32 logits per lane in the routing launch; T=8 routes in one
+# CTA (the few-slot launch of 8 warps), T=200 over several CTAs
+MANY = [
+    MoEConfig("many_e1000_t8", T=8, H=256, I=128, E=1000, k=8, bm=16, seed=110),
+    MoEConfig("many_e1000_t200", T=200, H=256, I=128, E=1000, k=8, bm=16, seed=111),
+    MoEConfig("many_e600_t16", T=16, H=256, I=128, E=600, k=6, bm=32, bias=True, seed=112),
+]
+
+
+@pytest.mark.parametrize("cfg", MANY, ids=lambda c: c.name)
+def test_forward_parity_many_experts(cuda_device, cfg):
+    d = make_layer(cfg)
+    g = _dev(d, cuda_device)
+    ref, ref_ids, ref_w = oracle.moe_forward(to_numpy(d["x"]), to_numpy(d["logits"]), cfg.k,
+                                             to_numpy(d["w13"]), to_numpy(d["w2"]), bias=to_numpy(d["bias"]))
+    layer = m.MoELayer(g["w13"], g["w2"], cfg.k, cfg.bm, out_dtype=torch.float32)
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=cuda_device)
+    tw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = layer(g["x"], g["logits"], g["bias"], topk_ids=ids, topk_w=tw, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.max(np.abs(tw.cpu().numpy() - ref_w)) <= 1e-6
+    assert_close(out.float().cpu().numpy(), ref, TOL_BF16, f"{cfg.name} out")
+
+
 SHARED = [
     # DeepSeek-style: selection-only bias and one shared expert
     MoEConfig("shared1", T=300, H=384, I=256, E=16, k=4, bm=32, bias=True, n_shared=1, bias_mode="select",
