@@ -304,6 +304,79 @@ __global__ void __launch_bounds__(kAlignThreads, 1) route_kernel(AlignParams p, 
   }
 }
 
+// Routing of at most 32 slots (decode: a few tokens), one CTA of 8 warps.
+// The same outputs as route_kernel<EPL, true, true> with one CTA, in fewer
+// steps: warps gate the tokens; warp 0 holds slot l in lane l, groups equal
+// expert ids with one match (the group size is the expert's count, the
+// lanes below in the group give the stable rank); the padded counts of all
+// E experts are scanned into segment offsets; block ids, sentinels and the
+// placement follow; the tile plan as in route_kernel.
+constexpr int kSmallRouteSlots = 32;
+constexpr int kSmallRouteThreads = 256;
+
+template <int EPL>
+__global__ void __launch_bounds__(kSmallRouteThreads, 1) route_small_kernel(AlignParams p, RouteExtra r) {
+  extern __shared__ int smem[];
+  const int E = p.E;
+  int* s_tot = smem;         // [E] slots per expert
+  int* s_off = s_tot + E;    // [E] padded counts, then segment offsets
+  int* s_g = s_off + E;      // [E] token groups per expert
+  int* sc = s_g + E;         // [3E + 2] scratch of finish_plan
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  for (int e = tid; e < E; e += blockDim.x) s_tot[e] = 0;
+  for (int t = warp; t < r.T; t += nwarps)
+    gate_token<EPL>(r.logits, r.bias, r.select_only != 0, t, r.E_routed, r.k, r.n_shared, r.ids_out, r.w_out,
+                    lane);
+  __syncthreads();   // the ids (global, written by this CTA) and the zeroed counts
+
+  // warp 0: slot `lane`'s expert, its stable rank among the slots of that expert
+  int key = -1, rank = 0;
+  if (warp == 0) {
+    key = lane < p.N ? __ldcg(p.ids + lane) : -1;
+    const bool bad = lane < p.N && (key < 0 || key >= E);
+    if (bad) key = -1;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) dev_flag(p.status, MOE_DEV_BAD_EXPERT_ID);
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    rank = __popc(peers & lanemask_lt());
+    if (key >= 0 && rank == 0) s_tot[key] = __popc(peers);   // one lane per expert
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) s_off[e] = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+  __syncthreads();   // the scan reads other threads' entries
+  const int total_post = block_exclusive_scan(s_off, E);
+  if (tid == 0) *p.num_post = total_post;
+
+  // block expert ids: the last expert whose segment starts at or before the block
+  const int nblk = total_post / p.bm;
+  for (int j = tid; j < nblk; j += blockDim.x) {
+    const int pos = j * p.bm;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= pos) lo = mid; else hi = mid - 1;
+    }
+    p.expert_ids[j] = lo;
+  }
+  // sentinel padding at the end of each touched expert's segment
+  for (int e = warp; e < E; e += nwarps) {
+    const int beg = s_off[e] + s_tot[e];
+    const int end = s_off[e] + (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+    for (int q = beg + lane; q < end; q += 32) p.sorted[q] = p.N;
+  }
+  if (warp == 0 && key >= 0) p.sorted[s_off[key] + rank] = lane;
+
+  // tile plan of the grouped GEMMs
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+    r.plan[plan_start(E) + e] = s_off[e];
+    r.plan[plan_rows(E) + e] = rows;
+    r.plan[plan_real(E) + e] = s_tot[e];
+    s_g[e] = (rows + r.tn - 1) / r.tn;
+  }
+  __syncthreads();
+  finish_plan(r.plan, s_g, E, r.nw_gu, r.nw_dn, r.tn, total_post, sc);
+}
+
 size_t align_smem_bytes(int E) { return (size_t)(kAlignWarps + 3) * E * sizeof(int); }
 
 template <typename K>
@@ -336,8 +409,23 @@ cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t strea
   return launch_route_impl(route_kernel<32, false, false>, p, r, grid, stream);
 }
 
+template <typename K>
+static cudaError_t launch_route_small(K kernel, const AlignParams& p, const RouteExtra& r, cudaStream_t stream) {
+  const size_t smem = (size_t)(6 * p.E + 2) * sizeof(int);   // <= 24.6 KB at E = 1024
+  kernel<<<1, kSmallRouteThreads, smem, stream>>>(p, r);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream) {
   const int epl = (p.E + 31) / 32;
+  if (p.N <= kSmallRouteSlots) {
+    if (epl <= 1) return launch_route_small(route_small_kernel<1>, p, r, stream);
+    if (epl <= 2) return launch_route_small(route_small_kernel<2>, p, r, stream);
+    if (epl <= 4) return launch_route_small(route_small_kernel<4>, p, r, stream);
+    if (epl <= 8) return launch_route_small(route_small_kernel<8>, p, r, stream);
+    if (epl <= 16) return launch_route_small(route_small_kernel<16>, p, r, stream);
+    return launch_route_small(route_small_kernel<32>, p, r, stream);
+  }
   if (epl <= 1) return launch_route_impl(route_kernel<1, true, true>, p, r, grid, stream);
   if (epl <= 2) return launch_route_impl(route_kernel<2, true, true>, p, r, grid, stream);
   if (epl <= 4) return launch_route_impl(route_kernel<4, true, true>, p, r, grid, stream);

@@ -25,8 +25,8 @@ SMALL = [
     MoEConfig("fewtok", T=3, H=1024, I=512, E=16, k=2, bm=16, seed=104),
     # many tokens per expert: 256-token tiles, several tiles per expert
     MoEConfig("manytok", T=1024, H=512, I=384, E=4, k=2, bm=64, seed=105),
-    # two tokens, four slots each: the forward fuses the combine and splits the
-    # down GEMM's K in two (few tiles)
+    # two tokens, four slots each: the forward fuses the combine, and routes
+    # its 8 slots with the few-slot routing kernel
     MoEConfig("tinybatch", T=2, H=512, I=512, E=16, k=4, bm=16, seed=109),
 ]
 
