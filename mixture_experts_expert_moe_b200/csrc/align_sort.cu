@@ -363,7 +363,8 @@ __global__ void __launch_bounds__(kSmallRouteThreads, 1) route_small_kernel(Alig
     const int end = s_off[e] + (s_tot[e] + p.bm - 1) / p.bm * p.bm;
     for (int q = beg + lane; q < end; q += 32) p.sorted[q] = p.N;
   }
-  if (warp == 0 && key >= 0) p.sorted[s_off[key] + rank] = lane;
+  if (warp == 0 && key >= 0 && MOE_IN_BOUNDS(s_off[key] + rank < p.N + p.E * (p.bm - 1), p.status))
+    p.sorted[s_off[key] + rank] = lane;
 
   // tile plan of the grouped GEMMs
   for (int e = tid; e < E; e += blockDim.x) {
