@@ -627,7 +627,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
     }
     line.update(extra)
-    print(json.dumps(line))
+    emit(line)
 
 
 # ---------------------------------------------------------------------------
@@ -776,7 +776,7 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     sample = (f"a batch of {n_tokens} seeded token per step of {workload_name(cfg, 'bf16')} through the "
               f"whole layer (float64 numpy on the host; the token's experts' weights held as float32)")
-    print(json.dumps({
+    emit({
         "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -784,7 +784,7 @@ def run_reference(args):
         "impl": "reference",
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }))
+    })
 
 
 def run_only(args):
@@ -802,13 +802,13 @@ def run_only(args):
                 cfg = cfg.with_(T=int(q[1:]))
             elif q.startswith("E"):
                 cfg = cfg.with_(E=int(q[1:]))
-        print(json.dumps(backward_report(m, cfg, steps, warmup, dev, pk)))
+        emit(backward_report(m, cfg, steps, warmup, dev, pk))
         return
     if parts[0] == "ep":          # ep_<config>: the expert-parallel layer over one rank
-        print(json.dumps(ep_report(m, CONFIGS[parts[1]], steps, warmup, dev)))
+        emit(ep_report(m, CONFIGS[parts[1]], steps, warmup, dev))
         return
     if parts[0] == "align":
-        print(json.dumps(align_report(m, dev, pk, int(parts[1]), iters=steps)))
+        emit(align_report(m, dev, pk, int(parts[1]), iters=steps))
         return
     if len(parts) > 2 and f"{parts[0]}_{parts[1]}" in CONFIGS:     # e.g. deepseek_shared
         parts = [f"{parts[0]}_{parts[1]}"] + parts[2:]
@@ -823,13 +823,38 @@ def run_only(args):
             cfg = cfg.with_(E=int(p[1:]))
         elif p.startswith("tn"):
             tile = int(p[2:])
+        elif p.startswith("H"):
+            cfg = cfg.with_(H=int(p[1:]))
+        elif p.startswith("I"):
+            cfg = cfg.with_(I=int(p[1:]))
         elif p == "bias":
             cfg = cfg.with_(bias=True)
     rep, _, _ = layer_report(m, cfg, steps, warmup, dev, pk, parts[1], tile_tokens=tile)
-    print(json.dumps(rep))
+    emit(rep)
+
+
+_OUT = sys.stdout
+
+
+def emit(obj):
+    """The run's one JSON line, on the process's original stdout."""
+    _OUT.write(json.dumps(obj) + "\n")
+    _OUT.flush()
+
+
+def _reserve_stdout():
+    """Send file descriptor 1 to stderr for the rest of the run, so that a
+    library writing to stdout (NCCL's version banner, for one) cannot put a
+    line next to the JSON line; returns a stream on the original stdout."""
+    sys.stdout.flush()
+    out = os.fdopen(os.dup(1), "w")
+    os.dup2(2, 1)
+    return out
 
 
 def main():
+    global _OUT
+    _OUT = _reserve_stdout()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
@@ -839,7 +864,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--only", default=None,
                     help="time one workload and print its report: <config>_<bf16|a8w8|mxfp8|mxfp4>"
-                         "[_bm<N>][_T<N>][_E<N>][_tn<N>] "
+                         "[_bm<N>][_T<N>][_E<N>][_H<N>][_I<N>][_tn<N>] "
                          "(configs: tiny, p5, deepseek, deepseek_shared, mixtral, decode) or align_<T>")
     args = ap.parse_args()
     if args.only:

@@ -92,3 +92,18 @@ def test_backward_accounting_by_hand():
     dw = E * 3 * H * I * 4                                     # fp32 gradients of every expert
     act = 2 * T * H * 2 + T * H * 4 + 2 * T * EL * 4           # x, dout in; dx out; logits in, dlogits out
     assert backward_bytes(T, H, I, E, touched, EL) == w_read + dw + act
+
+
+def test_bench_stdout_carries_only_the_json_line():
+    """Writes to file descriptor 1 by libraries (NCCL's version banner) and
+    stray prints go to stderr once bench.py has reserved stdout; the JSON
+    line alone reaches the original stdout."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import os, bench; bench._OUT = bench._reserve_stdout(); os.write(1, b'NCCL version x\\n'); "
+            "print('stray'); bench.emit({'metric': 'm', 'value': 1.0})")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout == '{"metric": "m", "value": 1.0}\n'
+    assert "NCCL version x" in r.stderr and "stray" in r.stderr
