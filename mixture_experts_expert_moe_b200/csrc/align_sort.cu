@@ -320,10 +320,14 @@ __global__ void __launch_bounds__(kSmallRouteThreads, 1) route_small_kernel(Alig
   const int E = p.E;
   int* s_tot = smem;         // [E] slots per expert
   int* s_off = s_tot + E;    // [E] padded counts, then segment offsets
-  int* s_g = s_off + E;      // [E] token groups per expert
+  int* s_g = s_off + E;      // [E] padded counts, then token groups per expert
   int* sc = s_g + E;         // [3E + 2] scratch of finish_plan
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   for (int e = tid; e < E; e += blockDim.x) s_tot[e] = 0;
+  if (r.zero_out) {   // in place of a memset launch
+    float4* z = reinterpret_cast<float4*>(r.zero_out);
+    for (long long i = tid; i < r.zero_n / 4; i += blockDim.x) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (int t = warp; t < r.T; t += nwarps)
     gate_token<EPL>(r.logits, r.bias, r.select_only != 0, t, r.E_routed, r.k, r.n_shared, r.ids_out, r.w_out,
                     lane);
@@ -341,7 +345,11 @@ __global__ void __launch_bounds__(kSmallRouteThreads, 1) route_small_kernel(Alig
     if (key >= 0 && rank == 0) s_tot[key] = __popc(peers);   // one lane per expert
   }
   __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) s_off[e] = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
+    s_off[e] = rows;
+    s_g[e] = rows;
+  }
   __syncthreads();   // the scan reads other threads' entries
   const int total_post = block_exclusive_scan(s_off, E);
   if (tid == 0) *p.num_post = total_post;
@@ -357,21 +365,17 @@ __global__ void __launch_bounds__(kSmallRouteThreads, 1) route_small_kernel(Alig
     }
     p.expert_ids[j] = lo;
   }
-  // sentinel padding at the end of each touched expert's segment
-  for (int e = warp; e < E; e += nwarps) {
-    const int beg = s_off[e] + s_tot[e];
-    const int end = s_off[e] + (s_tot[e] + p.bm - 1) / p.bm * p.bm;
-    for (int q = beg + lane; q < end; q += 32) p.sorted[q] = p.N;
-  }
   if (warp == 0 && key >= 0 && MOE_IN_BOUNDS(s_off[key] + rank < p.N + p.E * (p.bm - 1), p.status))
     p.sorted[s_off[key] + rank] = lane;
-
-  // tile plan of the grouped GEMMs
+  // per expert (one thread each): the sentinel padding at the end of its
+  // segment (at most block_size - 1 entries; none for most experts) and its
+  // entries of the tile plan
   for (int e = tid; e < E; e += blockDim.x) {
-    const int rows = (s_tot[e] + p.bm - 1) / p.bm * p.bm;
-    r.plan[plan_start(E) + e] = s_off[e];
+    const int start = s_off[e], real = s_tot[e], rows = s_g[e];
+    for (int q = start + real; q < start + rows; ++q) p.sorted[q] = p.N;
+    r.plan[plan_start(E) + e] = start;
     r.plan[plan_rows(E) + e] = rows;
-    r.plan[plan_real(E) + e] = s_tot[e];
+    r.plan[plan_real(E) + e] = real;
     s_g[e] = (rows + r.tn - 1) / r.tn;
   }
   __syncthreads();
@@ -417,9 +421,11 @@ static cudaError_t launch_route_small(K kernel, const AlignParams& p, const Rout
   return cudaGetLastError();
 }
 
+bool route_zeroes(long long N) { return N <= kSmallRouteSlots; }
+
 cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream) {
   const int epl = (p.E + 31) / 32;
-  if (p.N <= kSmallRouteSlots) {
+  if (route_zeroes(p.N)) {
     if (epl <= 1) return launch_route_small(route_small_kernel<1>, p, r, stream);
     if (epl <= 2) return launch_route_small(route_small_kernel<2>, p, r, stream);
     if (epl <= 4) return launch_route_small(route_small_kernel<4>, p, r, stream);

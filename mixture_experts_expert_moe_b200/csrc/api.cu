@@ -357,7 +357,8 @@ bool weights_ok(const FfnShape& s, const void* w13, const float* w13s, const voi
 // (s.E = E_routed + n_shared, s.k = k_routed + n_shared).
 moe_status_t run_route(const FfnShape& s, int n_shared, bool select_only, const float* logits, const float* bias,
                        int32_t* ids, float* w, int32_t* sorted, int32_t* expert_ids, int32_t* num_post,
-                       void* align_ws, int32_t* plan, int32_t* status, cudaStream_t stream) {
+                       void* align_ws, int32_t* plan, int32_t* status, cudaStream_t stream,
+                       float* zero_out = nullptr, long long zero_n = 0) {
   const int N = (int)s.N;
   int err = 0;
   const int max_ctas = moe::align_max_ctas(s.E, &err);
@@ -409,7 +410,18 @@ moe_status_t run_route(const FfnShape& s, int n_shared, bool select_only, const 
   r.tn = s.tn;
   r.nw_gu = s.I / 128;
   r.nw_dn = (s.H + 255) / 256;
-  if (grid > 1) MOE_CU(cudaMemsetAsync(p.barrier, 0, sizeof(int), stream));
+  r.zero_out = nullptr;
+  r.zero_n = 0;
+  if (zero_out) {
+    // the few-slot routing kernel zeroes the buffer; otherwise a memset does
+    if (moe::route_zeroes(N)) {
+      r.zero_out = zero_out;
+      r.zero_n = zero_n;
+    } else {
+      MOE_CU(cudaMemsetAsync(zero_out, 0, (size_t)zero_n * sizeof(float), stream));
+    }
+  }
+  if (grid > 1 && !moe::route_zeroes(N)) MOE_CU(cudaMemsetAsync(p.barrier, 0, sizeof(int), stream));
   MOE_CU(moe::launch_route(p, r, grid, stream));
   return MOE_OK;
 }
@@ -597,14 +609,15 @@ moe_status_t moe_forward(const moe_forward_args* a, void* ws, size_t ws_bytes, i
   float* out32 = !fused ? nullptr : out_bf16 ? reinterpret_cast<float*>(w + L.acc) : static_cast<float*>(a->out);
   float* y = fused ? nullptr : reinterpret_cast<float*>(w + L.y);
   MOE_CU(record(ev, 0, cs));
-  if (fused) MOE_CU(cudaMemsetAsync(out32, 0, (size_t)s.T * s.H * 4, cs));
   // gate, align&sort and the GEMM tile plan are one launch: stages 0..2 end together
   uint8_t* ffn_ws = w + L.ffn;
   int32_t* plan = reinterpret_cast<int32_t*>(ffn_ws + ffn_ws_layout(s).plan);
   {
     NvtxRange nr("moe: route (gate, align & sort, plan)");
+    // the fused combine's fp32 accumulator is zeroed by the routing step
     st = run_route(s, a->n_shared, a->bias_mode == MOE_BIAS_SELECT, a->logits, a->bias, ids, tw, sorted, eids,
-                   npost, w + L.align, plan, dev_status, cs);
+                   npost, w + L.align, plan, dev_status, cs, fused ? out32 : nullptr,
+                   fused ? (long long)s.T * s.H : 0);
   }
   if (st) return st;
   MOE_CU(record(ev, MOE_STAGE_GATE + 1, cs));

@@ -36,12 +36,17 @@ struct RouteExtra {
   float* w_out;         // [T*(k+n_shared)]
   int32_t* plan;        // plan layout below
   int tn, nw_gu, nw_dn;
+  float* zero_out;      // few-slot routing only (route_zeroes(N)): zeroes [zero_n] floats
+  long long zero_n;     // (a multiple of 4, 16-byte aligned), e.g. the fused combine's accumulator
 };
 
 size_t align_smem_bytes(int E);
 cudaError_t launch_align_sort(const AlignParams& p, int grid, cudaStream_t stream);
 // gate + align&sort + tile plan in one cooperative launch (p.chunk % (k + n_shared) == 0)
 cudaError_t launch_route(const AlignParams& p, const RouteExtra& r, int grid, cudaStream_t stream);
+// whether launch_route takes the few-slot kernel for N slots (which also
+// zeroes RouteExtra::zero_out)
+bool route_zeroes(long long N);
 int align_max_ctas(int E, int* err_out);
 cudaError_t launch_wait_timeout(int* counter, int32_t* status, long long timeout_ns, cudaStream_t stream);
 
