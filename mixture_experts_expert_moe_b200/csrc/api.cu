@@ -248,22 +248,23 @@ moe_status_t run_ffn(const FfnShape& s, const void* x, const FfnWeights& W, cons
                             status, stream));
   }
   MOE_CU(record(ev, MOE_STAGE_PLAN + 1, stream));
-  nvtxRangePushA("moe: gather");
-  if (s.mx) {
-    // every sorted row MX-quantises its token (codes + a scale per 32 elements)
-    MOE_CU(moe::launch_mx_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, reinterpret_cast<uint8_t*>(sA),
-                                     stream));
-  } else if (s.fp8 && N <= kFusedQuantSlots) {
-    // few slots: each sorted row quantises its token directly (one launch)
-    MOE_CU(moe::launch_quant_rows(x, sorted, /*gather=*/true, N, s.k, num_post, R, s.H, A, sA, status, stream));
-  } else if (s.fp8) {
-    // quantise each token once, then gather codes and scales into sorted order
-    MOE_CU(moe::launch_quant_rows(x, nullptr, false, N, s.k, nullptr, s.T, s.H, xq, sx, status, stream));
-    MOE_CU(moe::launch_gather_rows(xq, sx, sorted, num_post, R, N, s.k, s.H, A, sA, stream));
-  } else {
-    MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, R, N, s.k, s.H * 2, A, nullptr, stream));
+  {
+    NvtxRange nr_gather("moe: gather");
+    if (s.mx) {
+      // every sorted row MX-quantises its token (codes + a scale per 32 elements)
+      MOE_CU(moe::launch_mx_quant_rows(x, sorted, N, s.k, num_post, R, s.H, A, reinterpret_cast<uint8_t*>(sA),
+                                       stream));
+    } else if (s.fp8 && N <= kFusedQuantSlots) {
+      // few slots: each sorted row quantises its token directly (one launch)
+      MOE_CU(moe::launch_quant_rows(x, sorted, /*gather=*/true, N, s.k, num_post, R, s.H, A, sA, status, stream));
+    } else if (s.fp8) {
+      // quantise each token once, then gather codes and scales into sorted order
+      MOE_CU(moe::launch_quant_rows(x, nullptr, false, N, s.k, nullptr, s.T, s.H, xq, sx, status, stream));
+      MOE_CU(moe::launch_gather_rows(xq, sx, sorted, num_post, R, N, s.k, s.H, A, sA, stream));
+    } else {
+      MOE_CU(moe::launch_gather_rows(x, nullptr, sorted, num_post, R, N, s.k, s.H * 2, A, nullptr, stream));
+    }
   }
-  nvtxRangePop();
   MOE_CU(record(ev, MOE_STAGE_GATHER + 1, stream));
 
   moe::GemmLaunch g1 = {};
