@@ -25,6 +25,14 @@ GPUs) carries the exchange.  The split sizes of the variable all-to-alls are
 read on the host (one device-to-host copy of R counts per forward).  The
 per-rank steps are gathered in ``LibraryOps`` so that the exchange logic
 above is one function (``ep_forward``) whatever executes the steps.
+
+With ``chunks`` > 1 the rank's tokens are split into that many contiguous
+chunks that flow through the steps as a pipeline: the all-to-alls are
+issued asynchronously, so that the exchange of chunk c + 1 (and the return
+of chunk c - 1) proceed while the local experts compute chunk c (on GPUs:
+NCCL's stream next to the compute stream).  The split sizes of every chunk
+travel in one all-to-all up front.  Every rank must use the same number of
+chunks; a chunk may be empty on some rank.
 """
 from __future__ import annotations
 
@@ -72,9 +80,12 @@ def _all_to_all(send, send_counts, recv_counts, group):
     return recv
 
 
-def ep_forward(ops, x, logits, E, group=None, bias=None, bias_mode="logits"):
+def ep_forward(ops, x, logits, E, group=None, bias=None, bias_mode="logits", chunks=1):
     """One expert-parallel layer forward of this rank's tokens (module
-    docstring).  Every rank of ``group`` must call it, in the same order."""
+    docstring).  Every rank of ``group`` must call it, in the same order and
+    with the same ``chunks``."""
+    if chunks > 1:
+        return _ep_forward_pipelined(ops, x, logits, E, group, bias, bias_mode, chunks)
     R = dist.get_world_size(group)
     T, H = x.shape
     ids, w = ops.gate(logits, bias, bias_mode)
@@ -94,17 +105,85 @@ def ep_forward(ops, x, logits, E, group=None, bias=None, bias_mode="logits"):
     return ops.combine(y_slots, w)
 
 
+def _ep_forward_pipelined(ops, x, logits, E, group, bias, bias_mode, chunks):
+    """ep_forward over ``chunks`` contiguous token chunks, the exchanges of
+    neighbouring chunks overlapping the local experts' compute."""
+    R = dist.get_world_size(group)
+    T, H = x.shape
+    ids, w = ops.gate(logits, bias, bias_mode)
+    k = ids.shape[1]
+    bounds = [T * c // chunks for c in range(chunks + 1)]
+    routes = [ops.route(ids[bounds[c]:bounds[c + 1]], E, R) for c in range(chunks)]
+    # split sizes of every chunk in one exchange: send[r, c] slots of chunk c go to rank r
+    send_dev = torch.stack([torch.as_tensor(rt[1]).to(device=x.device, dtype=torch.int64).reshape(R)
+                            for rt in routes], dim=1).contiguous()
+    recv_dev = torch.empty_like(send_dev)
+    dist.all_to_all_single(recv_dev, send_dev, group=group)
+    send_c, recv_c = send_dev.cpu().tolist(), recv_dev.cpu().tolist()
+
+    def dispatch(c):
+        order, _, local = routes[c]
+        sc = [send_c[r][c] for r in range(R)]
+        rc = [recv_c[r][c] for r in range(R)]
+        rows_send = ops.permute(x[bounds[c]:bounds[c + 1]], order, k)
+        ids_send = local.reshape(-1, 1).contiguous()
+        rows = torch.empty((sum(rc), H), dtype=rows_send.dtype, device=x.device)
+        rids = torch.empty((sum(rc), 1), dtype=ids_send.dtype, device=x.device)
+        works = [dist.all_to_all_single(rows, rows_send, rc, sc, group=group, async_op=True),
+                 dist.all_to_all_single(rids, ids_send, rc, sc, group=group, async_op=True)]
+        return rows, rids, sc, rc, works, (rows_send, ids_send)
+
+    def compute(d):
+        rows, rids, sc, rc, works, _ = d
+        for wk in works:
+            wk.wait()
+        y = ops.expert_ffn(rows, rids.reshape(-1))
+        back = torch.empty((sum(sc), H), dtype=y.dtype, device=y.device)
+        return back, dist.all_to_all_single(back, y.contiguous(), sc, rc, group=group, async_op=True), y
+
+    def finish(c, b):
+        back, work, _ = b
+        work.wait()
+        tc = bounds[c + 1] - bounds[c]
+        if tc == 0:
+            return None
+        y_slots = ops.scatter(back, routes[c][0], tc * k)
+        return ops.combine(y_slots, w[bounds[c]:bounds[c + 1]])
+
+    sent = [None] * chunks
+    back = [None] * chunks
+    outs = []
+    sent[0] = dispatch(0)
+    if chunks > 1:
+        sent[1] = dispatch(1)
+    for c in range(chunks):
+        back[c] = compute(sent[c])
+        sent[c] = None
+        if c + 2 < chunks:
+            sent[c + 2] = dispatch(c + 2)
+        if c >= 1:
+            outs.append(finish(c - 1, back[c - 1]))
+            back[c - 1] = None
+    outs.append(finish(chunks - 1, back[chunks - 1]))
+    outs = [o for o in outs if o is not None]
+    if not outs:
+        return ops.combine(torch.empty((0, H), dtype=torch.float32, device=x.device), w)
+    return torch.cat(outs)
+
+
 class EPMoELayer:
     """The expert-parallel layer on this library's kernels: weights of this
     rank's E/R experts (bf16), top-k of the global E logits per token."""
 
-    def __init__(self, w13_local, w2_local, E, k, block_size, group=None, out_dtype=torch.bfloat16):
+    def __init__(self, w13_local, w2_local, E, k, block_size, group=None, out_dtype=torch.bfloat16, chunks=1):
         import mixture_experts_expert_moe_b200 as m
         R = dist.get_world_size(group)
         if E % R or w13_local.shape[0] != E // R:
             raise ValueError("the experts must split evenly: w13_local holds E / world_size experts")
-        self.E, self.group = E, group
+        if chunks < 1:
+            raise ValueError("chunks must be at least 1")
+        self.E, self.group, self.chunks = E, group, chunks
         self.ops = LibraryOps(m, w13_local, w2_local, k, block_size, out_dtype)
 
     def __call__(self, x, logits, bias=None, bias_mode="logits"):
-        return ep_forward(self.ops, x, logits, self.E, self.group, bias, bias_mode)
+        return ep_forward(self.ops, x, logits, self.E, self.group, bias, bias_mode, self.chunks)

@@ -71,10 +71,12 @@ class OracleOps:
 
     def combine(self, y_slots, w):
         import oracle
+        if w.shape[0] == 0:        # a rank without tokens
+            return torch.zeros(0, y_slots.shape[1], dtype=torch.float64)
         return torch.from_numpy(oracle.combine(y_slots.numpy(), w.numpy()))
 
 
-def _rank(rank, R, port, q):
+def _rank(rank, R, port, q, chunks=1, sizes=None):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=R)
     try:
@@ -82,20 +84,26 @@ def _rank(rank, R, port, q):
         x, logits, w13, w2 = _layer(R)
         El = E // R
         ops = OracleOps(w13[rank * El:(rank + 1) * El], w2[rank * El:(rank + 1) * El], K)
-        sl = slice(rank * T_PER_RANK, (rank + 1) * T_PER_RANK)
-        out = ep_forward(ops, torch.from_numpy(x[sl].copy()), torch.from_numpy(logits[sl].copy()), E)
+        sizes = sizes or [T_PER_RANK] * R      # tokens of each rank (a prefix of the layer's batch)
+        start = sum(sizes[:rank])
+        sl = slice(start, start + sizes[rank])
+        out = ep_forward(ops, torch.from_numpy(x[sl].copy()), torch.from_numpy(logits[sl].copy()), E,
+                         chunks=chunks)
         q.put((rank, out.numpy()))
     finally:
         dist.destroy_process_group()
 
 
+# chunks: 1 (one exchange), 3 (the pipelined exchange of 4-token chunks) and
+# 16 (more chunks than the rank's 12 tokens: empty chunks on every rank)
+@pytest.mark.parametrize("chunks", [1, 3, 16])
 @pytest.mark.parametrize("R", [2, 4])
-def test_ep_exchange_matches_single_process_layer(R):
+def test_ep_exchange_matches_single_process_layer(R, chunks):
     import oracle
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, R, port, q)) for r in range(R)]
+    procs = [ctx.Process(target=_rank, args=(r, R, port, q, chunks)) for r in range(R)]
     for p in procs:
         p.start()
     got = dict(q.get(timeout=120) for _ in range(R))
@@ -104,5 +112,28 @@ def test_ep_exchange_matches_single_process_layer(R):
         assert p.exitcode == 0
     x, logits, w13, w2 = _layer(R)
     ref, _, _ = oracle.moe_forward(x, logits, K, w13, w2)
+    out = np.concatenate([got[r] for r in range(R)])
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("chunks", [1, 3])
+def test_ep_exchange_uneven_ranks(chunks):
+    """Ranks with different token counts, one of them with none."""
+    import oracle
+    R, sizes = 4, [12, 7, 0, 5]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, R, port, q, chunks, sizes)) for r in range(R)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(R))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    x, logits, w13, w2 = _layer(R)
+    n = sum(sizes)
+    ref, _, _ = oracle.moe_forward(x[:n], logits[:n], K, w13, w2)
+    assert [got[r].shape[0] for r in range(R)] == sizes
     out = np.concatenate([got[r] for r in range(R)])
     np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)

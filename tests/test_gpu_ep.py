@@ -7,7 +7,8 @@
   library's kernels, the all-to-alls done by slicing the ranks' buffers in
   the order all_to_all_single uses (no rank waits on another), against the
   oracle layer;
-* EPMoELayer over a one-rank NCCL process group against the oracle layer.
+* EPMoELayer over a one-rank NCCL process group against the oracle layer,
+  with one exchange and with the pipelined exchange of 3 chunks.
 The exchange logic of ep_forward across several processes is covered on CPU
 with gloo ranks (tests/test_ep.py).
 """
@@ -100,11 +101,13 @@ def test_ep_layer_one_rank_nccl(cuda_device):
     try:
         cfg = CONFIGS["tiny"]
         d = make_layer(cfg, device=cuda_device)
-        layer = EPMoELayer(d["w13"], d["w2"], cfg.E, cfg.k, cfg.bm, out_dtype=torch.float32)
-        out = layer(d["x"], d["logits"])
-        torch.cuda.synchronize()
         ref, _, _ = oracle.moe_forward(to_numpy(d["x"]), to_numpy(d["logits"]), cfg.k, to_numpy(d["w13"]),
                                        to_numpy(d["w2"]))
-        assert_close(out.cpu().numpy(), ref, TOL_BF16, "EP layer, one NCCL rank")
+        # one exchange, and the pipelined exchange of 3 chunks (asynchronous all-to-alls)
+        for chunks in (1, 3):
+            layer = EPMoELayer(d["w13"], d["w2"], cfg.E, cfg.k, cfg.bm, out_dtype=torch.float32, chunks=chunks)
+            out = layer(d["x"], d["logits"])
+            torch.cuda.synchronize()
+            assert_close(out.cpu().numpy(), ref, TOL_BF16, f"EP layer, one NCCL rank, {chunks} chunk(s)")
     finally:
         dist.destroy_process_group()
