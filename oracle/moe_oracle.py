@@ -339,7 +339,8 @@ def combine(y, w):
     """out[t] = sum_j w[t, j] * y[t*k + j]  (float64)."""
     w = np.asarray(w, dtype=np.float64)
     T, k = w.shape
-    y = np.asarray(y, dtype=np.float64).reshape(T, k, -1)
+    y = np.asarray(y, dtype=np.float64)
+    y = y.reshape(T, k, y.shape[-1])      # rows t*k .. t*k+k-1 are token t's slots
     return np.einsum("tk,tkh->th", w, y)
 
 

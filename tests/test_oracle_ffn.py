@@ -172,6 +172,11 @@ def test_combine_against_loop():
         np.testing.assert_allclose(out[t], ref, rtol=1e-14)
 
 
+def test_combine_of_no_tokens():
+    out = mo.combine(np.zeros((0, 5)), np.zeros((0, 3)))
+    assert out.shape == (0, 5)
+
+
 def test_tokens_subset_matches_full():
     cfg, d = _layer()
     x, lg, w13, w2 = to_numpy(d["x"]), to_numpy(d["logits"]), to_numpy(d["w13"]), to_numpy(d["w2"])
