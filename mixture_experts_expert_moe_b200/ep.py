@@ -173,7 +173,9 @@ def _ep_forward_pipelined(ops, x, logits, E, group, bias, bias_mode, chunks):
 
 class EPMoELayer:
     """The expert-parallel layer on this library's kernels: weights of this
-    rank's E/R experts (bf16), top-k of the global E logits per token."""
+    rank's E/R experts (bf16), top-k of the global E logits per token.
+    ``chunks`` > 1 pipelines the rank's tokens through the exchange in that
+    many chunks (every rank of the group must use the same value)."""
 
     def __init__(self, w13_local, w2_local, E, k, block_size, group=None, out_dtype=torch.bfloat16, chunks=1):
         import mixture_experts_expert_moe_b200 as m
