@@ -86,6 +86,7 @@ constexpr int kFusedQuantSlots = 4096;
 // 37.9 us at 64 tokens per CTA, 29.7 at 32, 26.8 at 16; 25.2 us at 16 vs 38.5
 // at 64 for T = 256.
 constexpr int kRouteTokensPerCta = 16;
+constexpr long long kRouteZeroMaxFloats = 65536;   // 256 KB: a few us for one CTA
 
 bool align_args_ok(int T, int k, int E, int bm) {
   return T >= 0 && k >= 1 && E >= 1 && E <= 1024 && bm >= 1 && bm <= 1024 &&
@@ -414,8 +415,9 @@ moe_status_t run_route(const FfnShape& s, int n_shared, bool select_only, const 
   r.zero_out = nullptr;
   r.zero_n = 0;
   if (zero_out) {
-    // the few-slot routing kernel zeroes the buffer; otherwise a memset does
-    if (moe::route_zeroes(N)) {
+    // the few-slot routing kernel (one CTA) zeroes a small buffer; otherwise
+    // a memset does (spread over the GPU)
+    if (moe::route_zeroes(N) && zero_n <= kRouteZeroMaxFloats) {
       r.zero_out = zero_out;
       r.zero_n = zero_n;
     } else {

@@ -136,6 +136,28 @@ def test_forward_parity_many_experts(cuda_device, cfg):
     assert_close(out.float().cpu().numpy(), ref, TOL_BF16, f"{cfg.name} out")
 
 
+@pytest.mark.parametrize("a8w8", [False, True])
+def test_forward_parity_few_slots_wide_rows(cuda_device, a8w8):
+    """32 slots (the few-slot routing kernel) with the fused combine over a
+    token accumulator too large for that one-CTA kernel to zero (T*H > 65536
+    floats): the accumulator is cleared by a memset instead."""
+    cfg = MoEConfig("few_wide", T=4, H=16512, I=128, E=16, k=8, bm=16, seed=113).with_(a8w8=a8w8)
+    d = make_layer(cfg)
+    g = _dev(d, cuda_device)
+    w13, w2, s13, s2 = _weights(cfg, g)
+    ref, _, _ = oracle.moe_forward(
+        to_numpy(d["x"]), to_numpy(d["logits"]), cfg.k,
+        to_numpy(d["w13_q"] if a8w8 else d["w13"]), to_numpy(d["w2_q"] if a8w8 else d["w2"]),
+        a8w8=a8w8, w13_s=to_numpy(d.get("w13_s")), w2_s=to_numpy(d.get("w2_s")))
+    layer = m.MoELayer(w13, w2, cfg.k, cfg.bm, s13, s2, out_dtype=torch.float32)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    for _ in range(2):      # the second call must not add to the first one's sums
+        out = layer(g["x"], g["logits"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close(out.cpu().numpy(), ref, TOL_FP8 if a8w8 else TOL_BF16, "few slots, wide rows")
+
+
 SHARED = [
     # DeepSeek-style: selection-only bias and one shared expert
     MoEConfig("shared1", T=300, H=384, I=256, E=16, k=4, bm=32, bias=True, n_shared=1, bias_mode="select",
