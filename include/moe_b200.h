@@ -19,6 +19,13 @@
  *   combine  : out[t] = sum_j w[t,j] * y[t*k+j]                  (moe_combine)
  *   all four : moe_forward
  *
+ * Also: the layer's gradients (moe_backward), the per-rank steps of an
+ * expert-parallel layer (moe_ep_route, moe_permute_rows, moe_scatter_rows;
+ * the exchange between ranks is the caller's), MX block-scaled weights
+ * (moe_mx_tile_scales lays out their scales; moe_mx_quantize_rows is the
+ * activation quantiser), and align & sort without a caller workspace
+ * (moe_align_sort_noalloc).
+ *
  * Conventions (every entry point):
  *   - All tensor pointers are DEVICE pointers unless stated otherwise.  The
  *     caller owns every buffer and the stream; the library allocates no
